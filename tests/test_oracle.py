@@ -1,0 +1,338 @@
+"""Pins for the fp64 oracle: closed forms, invariants, brute force and a library
+special case.  None of these re-types the oracle's own formula; each is chosen
+so that a dropped term, a wrong sign, a wrong scale or a transposed index fails
+at least one of them.  CPU only."""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import ref
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+rng = np.random.default_rng(12345)
+
+
+def randn(*shape):
+    return rng.standard_normal(shape)
+
+
+# ---------------------------------------------------------------- closed forms
+def test_golden_identical_keys_causal():
+    with open(os.path.join(GOLDEN, "identical_keys_causal.json")) as f:
+        g = json.load(f)
+    o, lse = ref.attention(np.array(g["q"], float), np.array(g["k"], float),
+                           np.array(g["v"], float), causal=g["causal"])
+    np.testing.assert_allclose(o, np.array(g["expected_o"], float), rtol=0, atol=1e-14)
+    np.testing.assert_allclose(lse, np.array(g["expected_lse"], float), rtol=0, atol=1e-14)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_identical_keys_give_mean_of_v(causal):
+    S, H, dh = 37, 3, 8
+    q = randn(S, H, dh)
+    kvec = randn(1, H, dh)
+    k = np.repeat(kvec, S, axis=0)
+    v = randn(S, H, dh)
+    o, lse = ref.attention(q, k, v, causal=causal)
+    scale = 1 / math.sqrt(dh)
+    for i in range(S):
+        n = i + 1 if causal else S
+        for h in range(H):
+            np.testing.assert_allclose(o[i, h], v[:n, h].mean(axis=0), atol=1e-12)
+            s = scale * float(q[i, h] @ kvec[0, h])
+            assert abs(lse[h, i] - (s + math.log(n))) < 1e-12
+
+
+def test_causal_row_zero_is_v0():
+    S, H, dh = 16, 2, 16
+    q, k, v = randn(S, H, dh), randn(S, H, dh), randn(S, H, dh)
+    o, lse = ref.attention(q, k, v, causal=True)
+    np.testing.assert_allclose(o[0], v[0], atol=1e-14)
+    for h in range(H):
+        assert abs(lse[h, 0] - float(q[0, h] @ k[0, h]) / 4.0) < 1e-14
+
+
+def test_zero_queries_give_uniform_mean():
+    S, H, dh = 20, 2, 8
+    q = np.zeros((S, H, dh))
+    k, v = randn(S, H, dh), randn(S, H, dh)
+    o, lse = ref.attention(q, k, v, causal=True)
+    for i in range(S):
+        np.testing.assert_allclose(o[i], v[:i + 1].mean(axis=0), atol=1e-13)
+        np.testing.assert_allclose(lse[:, i], math.log(i + 1), atol=1e-14)
+
+
+def test_onehot_values_give_probabilities():
+    # V_j = e_j: O[i] is the probability row of query i: non-negative, sums to
+    # one, zero on keys the causal mask excludes.
+    S, dh = 32, 32
+    q, k = randn(S, 1, dh), randn(S, 1, dh)
+    v = np.eye(S).reshape(S, 1, dh)
+    o, _ = ref.attention(q, k, v, causal=True)
+    p = o[:, 0, :]
+    assert np.all(p >= 0)
+    np.testing.assert_allclose(p.sum(axis=1), 1.0, atol=1e-14)
+    assert np.all(np.triu(p, 1) == 0)
+
+
+def test_lse_bounds():
+    S, H, dh = 64, 2, 16
+    q, k, v = randn(S, H, dh), randn(S, H, dh), randn(S, H, dh)
+    _, lse = ref.attention(q, k, v, causal=True)
+    for h in range(H):
+        s = q[:, h] @ k[:, h].T / 4.0
+        for i in range(S):
+            mx = s[i, :i + 1].max()
+            assert mx - 1e-12 <= lse[h, i] <= mx + math.log(i + 1) + 1e-12
+
+
+# ------------------------------------------------------------- brute force
+def _scalar_attention(q, k, v, causal, scale, docs=None):
+    """Triple loop with math.exp, no numpy linear algebra."""
+    S, Hq, dh = q.shape
+    Hkv = k.shape[1]
+    o = [[[0.0] * dh for _ in range(Hq)] for _ in range(S)]
+    lse = [[-math.inf] * S for _ in range(Hq)]
+    for h in range(Hq):
+        g = h // (Hq // Hkv)
+        for i in range(S):
+            scores = []
+            for j in range(S):
+                if causal and j > i:
+                    continue
+                if docs is not None and docs[i] != docs[j]:
+                    continue
+                s = 0.0
+                for d in range(dh):
+                    s += float(q[i, h, d]) * float(k[j, g, d])
+                scores.append((j, s * scale))
+            if not scores:
+                continue
+            m = max(s for _, s in scores)
+            den = sum(math.exp(s - m) for _, s in scores)
+            for d in range(dh):
+                o[i][h][d] = sum(math.exp(s - m) * float(v[j, g, d]) for j, s in scores) / den
+            lse[h][i] = m + math.log(den)
+    return np.array(o), np.array(lse)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_bruteforce_gqa(causal):
+    S, Hq, Hkv, dh = 19, 4, 2, 5
+    q, k, v = randn(S, Hq, dh), randn(S, Hkv, dh), randn(S, Hkv, dh)
+    o, lse = ref.attention(q, k, v, causal=causal, row_block=7)
+    o2, lse2 = _scalar_attention(q, k, v, causal, 1 / math.sqrt(dh))
+    np.testing.assert_allclose(o, o2, atol=1e-12)
+    np.testing.assert_allclose(lse, lse2, atol=1e-12)
+
+
+def test_bruteforce_varlen():
+    S, H, dh = 24, 2, 4
+    cu = [0, 5, 6, 17, 24]
+    docs = [int(np.searchsorted(cu, i, side="right") - 1) for i in range(S)]
+    q, k, v = randn(S, H, dh), randn(S, H, dh), randn(S, H, dh)
+    o, lse = ref.attention(q, k, v, causal=True, cu_seqlens=cu)
+    o2, lse2 = _scalar_attention(q, k, v, True, 0.5, docs)
+    np.testing.assert_allclose(o, o2, atol=1e-12)
+    np.testing.assert_allclose(lse, lse2, atol=1e-12)
+
+
+def test_seq_equals_cp_size_one_token_per_rank():
+    # pwwt.cn Context Parallelism write-up §5.2: sequence length = CP size, one
+    # token per rank, checked element by element against a hand computation.
+    P = 4
+    dh = 3
+    q, k, v = randn(P, 1, dh), randn(P, 1, dh), randn(P, 1, dh)
+    o, lse = ref.ring_attention(q, k, v, P, P, "contiguous", causal=True)
+    o2, lse2 = _scalar_attention(q, k, v, True, 1 / math.sqrt(dh))
+    np.testing.assert_allclose(o, o2, atol=1e-13)
+    np.testing.assert_allclose(lse, lse2, atol=1e-13)
+
+
+# ------------------------------------------------------ library special case
+def test_matches_torch_sdpa_fp64_with_bool_mask():
+    S, Hq, Hkv, dh = 300, 4, 2, 32
+    q, k, v = randn(S, Hq, dh), randn(S, Hkv, dh), randn(S, Hkv, dh)
+    cu = [0, 40, 41, 200, 300]
+    o, lse = ref.attention(q, k, v, causal=True, cu_seqlens=cu)
+    docs = np.searchsorted(cu, np.arange(S), side="right") - 1
+    mask = (np.arange(S)[None, :] <= np.arange(S)[:, None]) & (docs[:, None] == docs[None, :])
+    tq = torch.from_numpy(q).permute(1, 0, 2)
+    tk = torch.from_numpy(k).permute(1, 0, 2).repeat_interleave(Hq // Hkv, dim=0)
+    tv = torch.from_numpy(v).permute(1, 0, 2).repeat_interleave(Hq // Hkv, dim=0)
+    ot = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=torch.from_numpy(mask))
+    np.testing.assert_allclose(o, ot.permute(1, 0, 2).numpy(), atol=1e-12)
+    s = torch.einsum("hqd,hkd->hqk", tq, tk) / math.sqrt(dh)
+    lt = torch.logsumexp(s.masked_fill(~torch.from_numpy(mask), -math.inf), dim=-1)
+    np.testing.assert_allclose(lse, lt.numpy(), atol=1e-12)
+
+
+# ------------------------------------------------------------- invariants
+@pytest.mark.parametrize("layout", ["contiguous", "zigzag"])
+@pytest.mark.parametrize("P", [1, 2, 4])
+@pytest.mark.parametrize("causal", [True, False])
+def test_split_then_merge_equals_unsplit(layout, P, causal):
+    # compassingai §二: the block recurrence is exact, so merging the P ring
+    # steps of every rank reproduces unsplit attention.
+    S, Hq, Hkv, dh = 48, 4, 2, 8
+    q, k, v = randn(S, Hq, dh), randn(S, Hkv, dh), randn(S, Hkv, dh)
+    o, lse = ref.attention(q, k, v, causal=causal)
+    o_r, lse_r = ref.ring_attention(q, k, v, S, P, layout, causal=causal)
+    order = np.concatenate([ref.shard_positions(S, P, layout, r) for r in range(P)])
+    np.testing.assert_allclose(o_r, o[order], atol=1e-12)
+    np.testing.assert_allclose(lse_r, lse[:, order], atol=1e-12)
+
+
+def test_split_invariance_varlen_zigzag():
+    S, H, dh, P = 64, 2, 8, 4
+    cu = [0, 3, 30, 31, 64]
+    q, k, v = randn(S, H, dh), randn(S, H, dh), randn(S, H, dh)
+    o, lse = ref.attention(q, k, v, causal=True, cu_seqlens=cu)
+    o_r, lse_r = ref.ring_attention(q, k, v, S, P, "zigzag", causal=True, cu_seqlens=cu)
+    order = ref.zigzag_order(S, P)
+    np.testing.assert_allclose(o_r, o[order], atol=1e-12)
+    np.testing.assert_allclose(lse_r, lse[:, order], atol=1e-12)
+
+
+def test_varlen_equals_separate_documents():
+    S, H, dh = 50, 2, 8
+    cu = [0, 7, 8, 33, 50]
+    q, k, v = randn(S, H, dh), randn(S, H, dh), randn(S, H, dh)
+    o, lse = ref.attention(q, k, v, causal=True, cu_seqlens=cu)
+    for a, b in zip(cu[:-1], cu[1:]):
+        od, ld = ref.attention(q[a:b], k[a:b], v[a:b], causal=True)
+        np.testing.assert_allclose(o[a:b], od, atol=1e-12)
+        np.testing.assert_allclose(lse[:, a:b], ld, atol=1e-12)
+
+
+def test_varlen_single_document_is_plain_causal():
+    S, H, dh = 40, 2, 8
+    q, k, v = randn(S, H, dh), randn(S, H, dh), randn(S, H, dh)
+    o1, l1 = ref.attention(q, k, v, causal=True)
+    o2, l2 = ref.attention(q, k, v, causal=True, cu_seqlens=[0, S])
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(l1, l2)
+
+
+def test_merge_edge_cases():
+    rows, H, dh = 5, 2, 3
+    o1, l1 = randn(rows, H, dh), randn(H, rows)
+    o, l = ref.lse_merge(o1[None], l1[None])
+    np.testing.assert_allclose(o, o1, atol=1e-15)
+    np.testing.assert_allclose(l, l1, atol=1e-15)
+    # a -inf partial with garbage O contributes nothing
+    bad = np.full_like(o1, np.nan)
+    o, l = ref.lse_merge(np.stack([o1, bad]), np.stack([l1, np.full_like(l1, -np.inf)]))
+    np.testing.assert_allclose(o, o1, atol=1e-15)
+    np.testing.assert_allclose(l, l1, atol=1e-15)
+    # two equal partials: same O, LSE + ln 2
+    o, l = ref.lse_merge(np.stack([o1, o1]), np.stack([l1, l1]))
+    np.testing.assert_allclose(o, o1, atol=1e-14)
+    np.testing.assert_allclose(l, l1 + math.log(2), atol=1e-14)
+    # all -inf: zero output
+    o, l = ref.lse_merge(np.stack([o1, o1]), np.full((2, H, rows), -np.inf))
+    assert np.all(o == 0) and np.all(np.isneginf(l))
+
+
+# ------------------------------------------------------------- layouts
+def test_zigzag_order_by_hand():
+    # S=16, P=2: chunks of 4; rank 0 = chunks 0, 3; rank 1 = chunks 1, 2
+    assert list(ref.zigzag_order(16, 2)) == [0, 1, 2, 3, 12, 13, 14, 15, 4, 5, 6, 7, 8, 9, 10, 11]
+
+
+def test_zigzag_round_trip_and_permutation():
+    x = randn(64, 3, 2)
+    y = ref.zigzag_reorder(x, 4)
+    assert sorted(ref.zigzag_order(64, 4)) == list(range(64))
+    np.testing.assert_array_equal(ref.zigzag_restore(y, 4), x)
+    lse = randn(3, 64)
+    np.testing.assert_array_equal(ref.zigzag_restore(ref.zigzag_reorder(lse, 4, axis=1), 4, axis=1), lse)
+
+
+def test_ulysses_index_formula_by_loops():
+    P, n, H, dh = 3, 4, 6, 2
+    x = randn(P, n, H, dh)
+    y = ref.ulysses_seq_to_head(x, P)
+    hg = H // P
+    assert y.shape == (P, P * n, hg, dh)
+    for r in range(P):
+        for p in range(P):
+            for s in range(n):
+                for hh in range(hg):
+                    for d in range(dh):
+                        assert y[r, p * n + s, hh, d] == x[p, s, r * hg + hh, d]
+    np.testing.assert_array_equal(ref.ulysses_head_to_seq(y, P), x)
+    np.testing.assert_array_equal(ref.ulysses_seq_to_head(x[:1], 1)[0], x[0])
+
+
+def test_ulysses_composite_equals_attention():
+    # compassingai §三: permute seq->head, full-sequence attention per head
+    # block, permute back == attention on the unsplit sequence (GQA 4:2, P=2).
+    P, S, Hq, Hkv, dh = 2, 24, 4, 2, 4
+    q, k, v = randn(S, Hq, dh), randn(S, Hkv, dh), randn(S, Hkv, dh)
+    o, lse = ref.attention(q, k, v, causal=True)
+    n = S // P
+    qh = ref.ulysses_seq_to_head(q.reshape(P, n, Hq, dh), P)
+    kh = ref.ulysses_seq_to_head(k.reshape(P, n, Hkv, dh), P)
+    vh = ref.ulysses_seq_to_head(v.reshape(P, n, Hkv, dh), P)
+    oh = np.stack([ref.attention(qh[r], kh[r], vh[r], causal=True)[0] for r in range(P)])
+    back = ref.ulysses_head_to_seq(oh, P).reshape(S, Hq, dh)
+    np.testing.assert_allclose(back, o, atol=1e-12)
+
+
+# ------------------------------------------------------ work counts
+def test_live_pair_counts_closed_forms():
+    S = 96
+    assert ref.live_pair_count(S, causal=True) == S * (S + 1) // 2
+    assert ref.live_pair_count(S, causal=False) == S * S
+    cu = [0, 10, 11, 60, 96]
+    lens = np.diff(cu)
+    assert ref.live_pair_count(S, True, cu) == int(sum(L * (L + 1) // 2 for L in lens))
+
+
+def test_pair_classes_contiguous_and_zigzag():
+    S, P = 64, 4
+    n = S // P
+    cls = ref.pair_classes(S, P, "contiguous")
+    for (r, t), (j, live, tot) in cls.items():
+        assert j == (r - t) % P
+        assert live == (n * n if j < r else (n * (n + 1) // 2 if j == r else 0))
+    c = S // (2 * P)
+    cls = ref.pair_classes(S, P, "zigzag")
+    for (r, t), (j, live, tot) in cls.items():
+        assert live == (2 * c * c + c if j == r else 2 * c * c)
+
+
+# ------------------------------------------------- planted mistakes are caught
+def test_pins_catch_planted_mistakes(monkeypatch):
+    """Plant plausible mistakes in the oracle (on the CPU) and check that the
+    pins above fail for each."""
+    S, H, dh = 12, 1, 4
+    q = np.zeros((S, H, dh))
+    k, v = randn(S, H, dh), randn(S, H, dh)
+    good_o, _ = ref.attention(q, k, v, causal=True)
+
+    orig = ref.explicit_mask
+
+    def off_by_one(qpos, kpos, causal, cu_seqlens=None):
+        m = orig(qpos, kpos, causal, cu_seqlens)
+        if causal:
+            m &= np.asarray(kpos)[None, :] < np.asarray(qpos)[:, None] + 0  # drops the diagonal
+            m[:, 0] = True
+        return m
+
+    monkeypatch.setattr(ref, "explicit_mask", off_by_one)
+    bad_o, _ = ref.attention(q, k, v, causal=True)
+    monkeypatch.setattr(ref, "explicit_mask", orig)
+    # the zero-query closed form (uniform mean over keys 0..i) rejects it
+    assert not np.allclose(bad_o[3], v[:4].mean(axis=0), atol=1e-9)
+    np.testing.assert_allclose(good_o[3], v[:4].mean(axis=0), atol=1e-13)
+
+    # wrong scale (1/dh instead of 1/sqrt(dh)) is caught by causal row 0
+    q2, k2 = randn(S, H, dh), randn(S, H, dh)
+    _, lse_bad = ref.attention(q2, k2, v, causal=True, scale=1.0 / dh)
+    assert abs(lse_bad[0, 0] - float(q2[0, 0] @ k2[0, 0]) / 2.0) > 1e-6

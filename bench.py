@@ -1,0 +1,465 @@
+#!/usr/bin/env python
+"""Benchmark of the context-parallel exact attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one pass of the hot path over one batch of synthetic input that is
+already resident in HBM.  For the default workload (ring attention forward,
+S=32768, 32 heads, dh=128, P=4 contiguous causal shards, bf16) a step is the
+ring-step schedule, the block-attention launch over all live block pairs and
+the fp32 LSE merge, all through ``cp_ring_attn_fwd``; zigzag workloads add the
+zigzag reorder of Q, K, V and the inverse reorder of O and LSE; the Ulysses
+workload is seq->head transpose, per-group attention, head->seq transpose.
+
+The metric is causal-effective TFLOP/s (4 * dh * hq per admitted (q, k) pair,
+divided by the step time); the JSON line also carries the a2a-permute GB/s of
+the Ulysses transpose, the roofline of the dominant kernel, an end-to-end
+figure with host buffers, the CPU oracle baseline and the SM clocks.
+
+Under torchrun every rank runs its own independent problem (weak scaling; no
+data crosses GPUs), and the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ring-attn fwd TFLOP/s & % BF16 tensor peak; a2a-permute GB/s % HBM"
+
+# DRAM traffic per launch of the block-attention kernel from an ncu capture,
+# keyed by the hash of the kernel source it was taken on (null once the
+# kernel changes).  Filled from profiles/ summaries.
+ATTN_TRAFFIC = {}
+
+
+def src_hash(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+# ----------------------------------------------------------------- helpers
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(hbm_gbs=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sus=d["bf16_tflops_sustained"],
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sus=1400.0, source="fallback")
+
+
+class Clocks:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.15)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for n, val in zip(names, parts[5:9]):
+                    if val.lower().startswith("active"):
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_init():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, ws):
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------- workloads
+def make_workload(name):
+    from context_exact_attention_step_b200 import api, synth
+    cfg = dict(synth.CONFIGS[name])
+    S, hq, hkv, dh, P = cfg["S"], cfg["hq"], cfg["hkv"], cfg["dh"], cfg["P"]
+    dtype = torch.float32 if cfg["dtype"] == "fp32" else torch.bfloat16
+    q, k, v = synth.qkv(S, hq, hkv, dh, std=cfg["std"], dtype=dtype)
+    cu = None
+    if cfg.get("varlen"):
+        cu = synth.cu_seqlens_from_lengths(synth.doc_lengths(S, cfg["doc_lo"], cfg["doc_hi"])).tolist()
+    layout = cfg["layout"]
+    dev = torch.device("cuda")
+    w = dict(name=name, cfg=cfg, S=S, hq=hq, hkv=hkv, dh=dh, P=P, layout=layout, cu=cu, dtype=dtype)
+    w["pairs"] = api.count_live_pairs(S, True, cu)
+    w["flops"] = 4.0 * dh * hq * w["pairs"]
+    w["host"] = [t.pin_memory() for t in (q, k, v)]
+    qd, kd, vd = (t.to(dev) for t in (q, k, v))
+    w["in"] = (qd, kd, vd)
+    o = torch.empty((S, hq, dh), device=dev, dtype=torch.float32)
+    lse = torch.empty((hq, S), device=dev, dtype=torch.float32)
+    w["out"] = (o, lse)
+    if layout == "ulysses":
+        ws = torch.empty(api.ulysses_attn_workspace_size(S, hq, hkv, dh, P), device=dev, dtype=torch.uint8)
+
+        def step():
+            api.ulysses_attn_fwd(qd, kd, vd, P, True, o=o, lse=lse, workspace=ws)
+    else:
+        cu_dev = torch.tensor(cu, dtype=torch.int32, device=dev) if cu is not None else None
+        ws = torch.empty(max(256, api.ring_attn_workspace_size(S, hq, hkv, dh, P, layout, True, dtype, cu)),
+                         device=dev, dtype=torch.uint8)
+        if layout == "zigzag":
+            qz, kz, vz = (torch.empty_like(t) for t in (qd, kd, vd))
+            oz = torch.empty_like(o)
+            lz = torch.empty_like(lse)
+
+            def step():
+                api.zigzag_reorder(qd, P, out=qz)
+                api.zigzag_reorder(kd, P, out=kz)
+                api.zigzag_reorder(vd, P, out=vz)
+                api.ring_attn_fwd(qz, kz, vz, P, layout, True, cu, cu_dev, o=oz, lse=lz, workspace=ws)
+                api.zigzag_reorder(oz, P, inverse=True, out=o)
+                api.zigzag_reorder(lz, P, inverse=True, seq_dim=1, out=lse)
+        else:
+            def step():
+                api.ring_attn_fwd(qd, kd, vd, P, layout, True, cu, cu_dev, o=o, lse=lse, workspace=ws)
+    w["step"] = step
+    w["ws_bytes"] = ws.numel()
+    return w
+
+
+def time_steps(w, steps, warmup, ws):
+    from context_exact_attention_step_b200 import api
+    step = w["step"]
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    ab, ae, me = [ev() for _ in range(steps)], [ev() for _ in range(steps)], [ev() for _ in range(steps)]
+    for e in ab + ae + me:
+        e.record()  # creates the CUDA handles
+    torch.cuda.synchronize()
+    barrier(ws)
+    torch.cuda.synchronize()
+    t0, t1 = ev(), ev()
+    n0 = api.kernel_launch_count()
+    t0.record()
+    for i in range(steps):
+        api.set_profile_events(ab[i], ae[i], me[i])
+        step()
+    t1.record()
+    api.set_profile_events(None, None, None)
+    torch.cuda.synchronize()
+    launches = api.kernel_launch_count() - n0
+    barrier(ws)
+    total_ms = t0.elapsed_time(t1)
+    attn_ms = [a.elapsed_time(b) for a, b in zip(ab, ae)]
+    merge_ms = [a.elapsed_time(b) for a, b in zip(ae, me)] if w["layout"] != "ulysses" else []
+    err = api.device_error()
+    if err:
+        raise RuntimeError(f"device error word {err:#x}: a kernel gave up waiting")
+    return total_ms, attn_ms, merge_ms, launches
+
+
+def time_e2e(w, steps):
+    """Same step through the public API with host buffers: pinned host Q, K, V
+    copied in and O, LSE copied out inside the timed region."""
+    qh, kh, vh = w["host"]
+    qd, kd, vd = w["in"]
+    o, lse = w["out"]
+    oh = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    lh = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+
+    def one():
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        w["step"]()
+        oh.copy_(o, non_blocking=True)
+        lh.copy_(lse, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        one()
+    t1.record()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / steps
+    h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
+    d2h = oh.numel() * oh.element_size() + lh.numel() * lh.element_size()
+    return ms, h2d, d2h
+
+
+def time_permute(reps=20):
+    """a2a-permute GB/s of the Ulysses transposes on the 128K-token GQA
+    workload: seq->head of Q (32 heads), K and V (8 heads), head->seq of the
+    fp32 O; bytes = read + write of every element once."""
+    from context_exact_attention_step_b200 import api, synth
+    S, hq, hkv, dh, P = 131072, 32, 8, 128, 8
+    dev = torch.device("cuda")
+    q = synth.normal((S, hq, dh), 1, 0.5).to(dev)
+    k = synth.normal((S, hkv, dh), 2, 0.5).to(dev)
+    v = synth.normal((S, hkv, dh), 3, 0.5).to(dev)
+    oh = torch.randn((P, S, hq // P, dh), device=dev, dtype=torch.float32)
+    qh = torch.empty((P, S, hq // P, dh), device=dev, dtype=torch.bfloat16)
+    kh = torch.empty((P, S, hkv // P, dh), device=dev, dtype=torch.bfloat16)
+    vh = torch.empty_like(kh)
+    o = torch.empty((S, hq, dh), device=dev, dtype=torch.float32)
+
+    def run():
+        api.ulysses_permute(q, P, "seq_to_head", out=qh)
+        api.ulysses_permute(k, P, "seq_to_head", out=kh)
+        api.ulysses_permute(v, P, "seq_to_head", out=vh)
+        api.ulysses_permute(oh, P, "head_to_seq", out=o)
+
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(reps):
+        run()
+    t1.record()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / reps
+    nbytes = 2 * sum(t.numel() * t.element_size() for t in (q, k, v, oh))
+    return dict(gbs=nbytes / (ms * 1e-3) / 1e9, ms=ms, bytes=nbytes)
+
+
+# ----------------------------------------------------------------- CPU oracle
+def oracle_sample_rate(w, target_s=12.0, max_rows=1024, seed=0):
+    """Times the fp64 oracle on a bounded sample of the same workload: batches
+    of 32 query rows (natural positions, seeded) against every key, all heads.
+    Returns causal-effective TFLOP/s of the sample and what was sampled."""
+    from oracle import ref
+    from context_exact_attention_step_b200 import synth
+    q, k, v = (t.to(torch.float64).numpy() for t in synth.qkv(w["S"], w["hq"], w["hkv"], w["dh"],
+                                                                 std=w["cfg"]["std"], dtype=w["dtype"]))
+    if w["dtype"] == torch.float32:  # the kernel consumes bf16-rounded values
+        q, k, v = (torch.from_numpy(t).to(torch.bfloat16).double().numpy() for t in (q, k, v))
+    rng = np.random.default_rng(seed)
+    cu = w["cu"]
+    t_total, flops, rows_done = 0.0, 0.0, 0
+    while t_total < target_s and rows_done < max_rows:
+        rows = np.sort(rng.integers(0, w["S"], 32))
+        t0 = time.perf_counter()
+        ref.attention(q[rows], k, v, causal=True, cu_seqlens=cu, qpos=rows)
+        t_total += time.perf_counter() - t0
+        if cu is None:
+            live = (rows + 1).sum()
+        else:
+            starts = np.asarray(cu)[np.searchsorted(cu, rows, side="right") - 1]
+            live = (rows - starts + 1).sum()
+        flops += 4.0 * w["dh"] * w["hq"] * float(live)
+        rows_done += 32
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    return dict(value=flops / t_total / 1e12, unit="TFLOP/s", cores=cores, kind="oracle",
+                sample=f"{rows_done} query rows (seeded, uniform positions) x all {w['S']} keys x {w['hq']} heads, "
+                       f"fp64 numpy, {t_total:.1f} s")
+
+
+# ----------------------------------------------------------------- arms
+def run_reference(args, ws, rank):
+    """Reference arm: the fp64 CPU oracle as it stands, on the same workload,
+    metric and unit; every step is a bounded sample of 32 query rows."""
+    if rank != 0:
+        return
+    from context_exact_attention_step_b200 import synth
+    from oracle import ref
+    name = args.workload
+    cfg = synth.CONFIGS[name]
+    S, hq, hkv, dh = cfg["S"], cfg["hq"], cfg["hkv"], cfg["dh"]
+    dtype = torch.float32 if cfg["dtype"] == "fp32" else torch.bfloat16
+    q, k, v = (t.to(torch.bfloat16).double().numpy() for t in synth.qkv(S, hq, hkv, dh, std=cfg["std"], dtype=dtype))
+    cu = None
+    if cfg.get("varlen"):
+        cu = synth.cu_seqlens_from_lengths(synth.doc_lengths(S, cfg["doc_lo"], cfg["doc_hi"])).tolist()
+    rng = np.random.default_rng(1)
+    rows_per_step = 32
+
+    def step():
+        rows = np.sort(rng.integers(0, S, rows_per_step))
+        ref.attention(q[rows], k, v, causal=True, cu_seqlens=cu, qpos=rows)
+        if cu is None:
+            return float((rows + 1).sum())
+        starts = np.asarray(cu)[np.searchsorted(cu, rows, side="right") - 1]
+        return float((rows - starts + 1).sum())
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    live = sum(step() for _ in range(args.steps))
+    dt = time.perf_counter() - t0
+    val = 4.0 * dh * hq * live / dt / 1e12
+    cores = len(os.sched_getaffinity(0))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": name, **{k_: cfg[k_] for k_ in ("S", "hq", "hkv", "dh", "P", "layout")}},
+        "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{rows_per_step} seeded query rows x all keys x all heads per step"},
+        "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, ws, rank, local):
+    from context_exact_attention_step_b200 import api
+    from context_exact_attention_step_b200 import build as _build
+    _build.build()
+    pk = peaks()
+    w = make_workload(args.workload)
+    clocks = Clocks(local)
+    clocks.start()
+    total_ms, attn_ms, merge_ms, launches = time_steps(w, args.steps, args.warmup, ws)
+    ck = clocks.stop()
+    ms_step = max_over_ranks(total_ms / args.steps, ws)
+    value = w["flops"] * ws / (ms_step * 1e-3) / 1e12
+    attn_avg = statistics.mean(attn_ms)
+    attn_tf = w["flops"] / (attn_avg * 1e-3) / 1e12
+    traffic = ATTN_TRAFFIC.get(src_hash(os.path.join(ROOT, "context_exact_attention_step_b200", "csrc",
+                                                     "attn_fwd.cu")))
+    e2e_ms, h2d, d2h = time_e2e(w, args.e2e_steps)
+    e2e_ms = max_over_ranks(e2e_ms, ws)
+    perm = time_permute() if not args.no_permute else None
+    cfg = w["cfg"]
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w["name"], "S": w["S"], "hq": w["hq"], "hkv": w["hkv"], "dh": w["dh"], "P": w["P"],
+                   "layout": w["layout"], "causal": True, "input_dtype": cfg["dtype"],
+                   "admitted_pairs": w["pairs"], "flops_per_step": w["flops"],
+                   "l2": "inputs larger than L2 (Q+K+V %.0f MB, partials %.0f MB)" % (
+                       sum(t.numel() * t.element_size() for t in w["in"]) / 1e6, w["ws_bytes"] / 1e6),
+                   "per_gpu": "independent problem per GPU"},
+        "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel", "achieved": attn_tf, "peak": pk["bf16"],
+                     "unit": "TFLOP/s", "frac": attn_tf / pk["bf16"], "traffic": traffic,
+                     "peak_source": pk["source"] + " burst bf16", "frac_of_sustained": attn_tf / pk["bf16_sus"],
+                     "frac_of_nominal_2250": attn_tf / 2250.0, "attn_ms": attn_avg},
+        "e2e": {"value": w["flops"] * ws / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": int(launches),
+        "clocks": ck,
+    }
+    if merge_ms:
+        mb = merge_bytes(w)
+        mms = statistics.mean(merge_ms)
+        line["merge"] = {"ms": mms, "gbs": mb / (mms * 1e-3) / 1e9, "frac_hbm": mb / (mms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                         "bytes": mb}
+    if perm:
+        line["a2a_permute"] = {"gbs": perm["gbs"], "frac_hbm": perm["gbs"] / pk["hbm_gbs"], "ms": perm["ms"],
+                               "bytes": perm["bytes"], "workload": "ulysses_gqa_128k Q,K,V seq->head + fp32 O head->seq"}
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_sample_rate(w)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def merge_bytes(w):
+    """Algorithmic bytes of the merge: every live partial (O fp32 + LSE) read
+    once, the output O and LSE written once."""
+    from context_exact_attention_step_b200 import api
+    sch = api.ring_schedule(w["S"], w["P"], w["layout"], True, w["cu"])
+    rows = int(sch["q_rows"].sum())
+    per_row = w["hq"] * (w["dh"] + 1) * 4
+    return rows * per_row + w["S"] * per_row
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--workload", default="ring_contig_32k")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-permute", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), rank)
+        return
+    ws, rank, local = dist_init()
+    try:
+        run_ours(args, ws, rank, local)
+    finally:
+        if ws > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

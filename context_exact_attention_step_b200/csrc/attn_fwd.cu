@@ -1,0 +1,514 @@
+// Block attention forward for one launch of ring-step block pairs (sm_100a).
+//
+// For every block pair of the plan, every query head and every 256-row query
+// tile, one CTA computes the partial result of those queries against the
+// pair's key/value rows:
+//     S = Q K^T * scale, masked by global position (causal: k <= q;
+//     document mask: same document), online softmax over the key tiles,
+//     O = softmax(S) V normalised within the pair, LSE = ln sum exp(S).
+// This is the per-block recurrence of the "序列並行（Sequence Parallelism）"
+// concept page (compassingai), 技術原理 §二 "Ring Attention 的塊級線上
+// Softmax" (running max m, running denominator l, rescaled O; S = Q K^T /
+// sqrt(d_k)), with the mask offsets of the "Context Parallelism" write-up
+// (pwwt.cn) §3.3 taken from each block's global positions.
+//
+// CTA layout (384 threads, one CTA per SM):
+//   warp 0      TMA producer: Q tile once, then K/V tiles into a 4-stage ring
+//   warp 1      tcgen05.mma issuer (one thread) and TMEM owner
+//   warps 2-3   idle
+//   warps 4-7   softmax of query sub-tile 0 (rows 0-127; one row per thread)
+//   warps 8-11  softmax of query sub-tile 1 (rows 128-255)
+// TMEM (512 columns): S0 | S1 (128 fp32 columns each; P is written back over
+// S as packed bf16) | O0 | O1 (dh columns each).
+// Tensor-pipe order per key tile j: PV0(j), S0(j+1), PV1(j), S1(j+1), so
+// each sub-tile's softmax overlaps the other sub-tile's MMAs.
+// Rescaling of O is lazy: the running max used for P only moves when the tile
+// max exceeds it by more than 2^8, which keeps P <= 256 and the result exact.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math_constants.h>
+
+#include <atomic>
+
+#include "plan.h"
+#include "sm100_ptx.cuh"
+
+namespace cp {
+
+std::atomic<uint64_t>& launch_counter();
+
+__device__ uint32_t g_attn_err = 0;
+
+constexpr int kThreads = 384;
+constexpr int kLoNone = -(1 << 30);
+constexpr int kHiNone = (1 << 30);
+
+template <int DH>
+struct AttnCfg {
+  static constexpr int kBoxes = DH / 64;            // 128-byte column boxes per row
+  static constexpr int kBoxBytes = 128 * 128;       // 128 rows x 128 bytes
+  static constexpr int kTileBytes = kBoxes * kBoxBytes;
+  static constexpr int kStages = DH == 128 ? 4 : 8;
+  static constexpr int kQBytes = 2 * kTileBytes;
+  static constexpr int kBarBytes = 256;
+  static constexpr int kSmemBytes = 1024 + kQBytes + kStages * kTileBytes + kBarBytes;
+  static constexpr uint32_t kTmemCols = 512;
+  // TMEM column of the S/P tile and of the O accumulator of sub-tile t
+  __device__ static constexpr uint32_t col_s(int t) { return (uint32_t)t * 128u; }
+  __device__ static constexpr uint32_t col_o(int t) { return 256u + (uint32_t)t * DH; }
+};
+
+struct KTile {
+  int buf_row, pos, valid;
+  bool live0, live1;
+};
+
+// Enumerates the key tiles of a block pair that are not fully masked for at
+// least one of the two query sub-tiles.  Every role of the CTA runs its own
+// copy, so all of them see the same sequence without communicating.
+struct KIter {
+  const cp_pair_desc* pd;
+  int seg, t;
+  int vis_lo[2], vis_hi[2];
+  bool alive[2];
+
+  __device__ bool next(KTile& out) {
+    while (seg < pd->nk) {
+      const int len = pd->k[seg].len;
+      const int off = t * CP_KV_TILE;
+      if (off >= len) {
+        ++seg;
+        t = 0;
+        continue;
+      }
+      const int ka = pd->k[seg].pos + off;
+      // Positions grow along a segment: once past both causal limits, the
+      // rest of the segment is masked.
+      if ((!alive[0] || ka > vis_hi[0]) && (!alive[1] || ka > vis_hi[1])) {
+        ++seg;
+        t = 0;
+        continue;
+      }
+      ++t;
+      const int valid = min(CP_KV_TILE, len - off);
+      const int kb = ka + valid - 1;
+      const bool l0 = alive[0] && kb >= vis_lo[0] && ka <= vis_hi[0];
+      const bool l1 = alive[1] && kb >= vis_lo[1] && ka <= vis_hi[1];
+      if (l0 || l1) {
+        out.buf_row = pd->k[seg].buf_row + off;
+        out.pos = ka;
+        out.valid = valid;
+        out.live0 = l0;
+        out.live1 = l1;
+        return true;
+      }
+    }
+    return false;
+  }
+};
+
+__device__ __forceinline__ int doc_start(const int32_t* __restrict__ cu, int n_docs, int x) {
+  int lo = 0, hi = n_docs - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(cu + mid) <= x) lo = mid; else hi = mid - 1;
+  }
+  return __ldg(cu + lo);
+}
+
+struct Item {
+  const cp_pair_desc* pd;
+  int h, hk;
+  int q_buf_row0, q_pos0, q_valid, out_row0;
+  // per query sub-tile: visible window hull and the fully-visible window
+  int vis_lo[2], vis_hi[2], full_lo[2], full_hi[2];
+  bool alive[2];
+};
+
+__device__ __forceinline__ void decode_item(const cp_attn_plan& plan, Item& it) {
+  const int cta = blockIdx.x;
+  int p = 0;
+  while (p + 1 < plan.n_pairs && plan.pairs[p + 1].cta_begin <= cta) ++p;
+  const cp_pair_desc* pd = &plan.pairs[p];
+  const int local = cta - pd->cta_begin;
+  it.pd = pd;
+  it.h = local / pd->qtiles;
+  it.hk = it.h / (plan.hq / plan.hkv);
+  int qt = local - it.h * pd->qtiles;
+  if (pd->reverse) qt = pd->qtiles - 1 - qt;
+  int s = 0;
+  for (; s < pd->nq; ++s) {
+    const int nt = (pd->q[s].len + CP_Q_TILE - 1) / CP_Q_TILE;
+    if (qt < nt) break;
+    qt -= nt;
+  }
+  const int off = qt * CP_Q_TILE;
+  it.q_buf_row0 = pd->q[s].buf_row + off;
+  it.q_pos0 = pd->q[s].pos + off;
+  it.q_valid = min(CP_Q_TILE, pd->q[s].len - off);
+  it.out_row0 = pd->q[s].out_row + off;
+  for (int t = 0; t < 2; ++t) {
+    const int vt = min(128, it.q_valid - t * 128);
+    it.alive[t] = vt > 0;
+    const int qa = it.q_pos0 + t * 128;
+    const int qb = qa + max(vt, 1) - 1;
+    const bool varlen = plan.n_docs > 0;
+    it.vis_lo[t] = varlen ? doc_start(plan.cu_seqlens, plan.n_docs, qa) : kLoNone;
+    it.full_lo[t] = varlen ? doc_start(plan.cu_seqlens, plan.n_docs, qb) : kLoNone;
+    it.vis_hi[t] = plan.causal ? qb : kHiNone;
+    it.full_hi[t] = plan.causal ? qa : kHiNone;
+  }
+}
+
+__device__ __forceinline__ void make_iter(const Item& it, KIter& ki) {
+  ki.pd = it.pd;
+  ki.seg = 0;
+  ki.t = 0;
+  for (int t = 0; t < 2; ++t) {
+    ki.vis_lo[t] = it.vis_lo[t];
+    ki.vis_hi[t] = it.vis_hi[t];
+    ki.alive[t] = it.alive[t];
+  }
+}
+
+template <int DH>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ cp_attn_plan plan) {
+  using C = AttnCfg<DH>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sKV = smem + C::kQBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + C::kStages * C::kTileBytes);
+  // barrier indices
+  const int B_Q = 0, B_FULL = 1, B_EMPTY = 1 + C::kStages, B_S = 1 + 2 * C::kStages, B_P = B_S + 2,
+            B_O = B_P + 2, B_DRAIN = B_O + 2, B_COUNT = B_DRAIN + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + B_COUNT);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  auto bar = [&](int i) { return smem_addr(bars + i); };
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  uint32_t* err = plan.err;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(B_Q), 1);
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(bar(B_FULL + s), 1);
+      mbar_init(bar(B_EMPTY + s), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(B_S + t), 1);
+      mbar_init(bar(B_P + t), 128);
+      mbar_init(bar(B_O + t), 1);
+    }
+    mbar_init(bar(B_DRAIN), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(tmem_holder), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  Item it;
+  decode_item(plan, it);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar(B_Q), C::kQBytes);
+      for (int t = 0; t < 2; ++t)
+        for (int b = 0; b < C::kBoxes; ++b)
+          tma_load_2d(smem_addr(sQ + (t * C::kBoxes + b) * C::kBoxBytes), &tm_q, it.h * DH + b * 64,
+                      it.q_buf_row0 + t * 128, bar(B_Q));
+      KIter ki;
+      make_iter(it, ki);
+      KTile kt;
+      uint32_t c = 0;
+      bool ok = true;
+      while (ok && ki.next(kt)) {
+        for (int w = 0; w < 2 && ok; ++w) {
+          const int slot = c % C::kStages;
+          const uint32_t ph = (c / C::kStages) & 1u;
+          ok = mbar_wait(bar(B_EMPTY + slot), ph ^ 1u, abort_flag, err);
+          if (!ok) break;
+          mbar_arrive_expect_tx(bar(B_FULL + slot), C::kTileBytes);
+          const CUtensorMap* m = w == 0 ? &tm_k : &tm_v;
+          for (int b = 0; b < C::kBoxes; ++b)
+            tma_load_2d(smem_addr(sKV + slot * C::kTileBytes + b * C::kBoxBytes), m, it.hk * DH + b * 64,
+                        kt.buf_row, bar(B_FULL + slot));
+          ++c;
+        }
+      }
+      // Drain: make sure every copy this thread issued has landed before the
+      // CTA can exit (only matters after an abort).
+      const uint32_t first = c > (uint32_t)C::kStages ? c - C::kStages : 0u;
+      for (uint32_t i = first; i < c; ++i)
+        mbar_wait(bar(B_FULL + i % C::kStages), (i / C::kStages) & 1u, abort_flag, nullptr, 1000000000ull);
+      mbar_wait(bar(B_Q), 0, abort_flag, nullptr, 1000000000ull);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, DH, true);
+      const uint32_t sq_base = smem_addr(sQ);
+      const uint32_t skv_base = smem_addr(sKV);
+      auto issue_s = [&](int t, int slot) {
+#pragma unroll
+        for (int kk = 0; kk < DH / 16; ++kk) {
+          const uint32_t box = kk >> 2, koff = (kk & 3) * 32;
+          const uint64_t a =
+              sdesc_sw128(sq_base + (t * C::kBoxes + box) * C::kBoxBytes + koff, 16, 1024);
+          const uint64_t b = sdesc_sw128(skv_base + slot * C::kTileBytes + box * C::kBoxBytes + koff, 16, 1024);
+          tc_mma_ss(tmem + C::col_s(t), a, b, idesc_qk, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int t, int slot, bool acc) {
+#pragma unroll
+        for (int kk = 0; kk < CP_KV_TILE / 16; ++kk) {
+          const uint64_t b = sdesc_sw128(skv_base + slot * C::kTileBytes + kk * 2048, C::kBoxBytes, 1024);
+          tc_mma_ts(tmem + C::col_o(t), tmem + C::col_s(t) + kk * 8, b, idesc_pv, (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      auto kslot = [&](int j) { return (2 * j) % C::kStages; };
+      auto kph = [&](int j) { return (uint32_t)(((2 * j) / C::kStages) & 1); };
+      auto vslot = [&](int j) { return (2 * j + 1) % C::kStages; };
+      auto vph = [&](int j) { return (uint32_t)(((2 * j + 1) / C::kStages) & 1); };
+
+      bool ok = mbar_wait(bar(B_Q), 0, abort_flag, err);
+      KIter ki;
+      make_iter(it, ki);
+      KTile cur, nxt;
+      bool have = ok && ki.next(cur);
+      uint32_t pc[2] = {0u, 0u};
+      bool acc[2] = {false, false};
+      int j = 0;
+      if (have) {
+        ok = mbar_wait(bar(B_FULL + kslot(0)), kph(0), abort_flag, err);
+        if (ok) {
+          tc_fence_after();
+          if (cur.live0) { issue_s(0, kslot(0)); tc_commit(bar(B_S + 0)); }
+          if (cur.live1) { issue_s(1, kslot(0)); tc_commit(bar(B_S + 1)); }
+          tc_commit(bar(B_EMPTY + kslot(0)));
+        }
+        have = ok;
+      }
+      while (have) {
+        const bool hn = ki.next(nxt);
+        if (!(ok = mbar_wait(bar(B_FULL + vslot(j)), vph(j), abort_flag, err))) break;
+        if (cur.live0) {
+          if (!(ok = mbar_wait(bar(B_P + 0), pc[0] & 1u, abort_flag, err))) break;
+          ++pc[0];
+          tc_fence_after();
+          issue_pv(0, vslot(j), acc[0]);
+          acc[0] = true;
+        }
+        if (hn) {
+          if (!(ok = mbar_wait(bar(B_FULL + kslot(j + 1)), kph(j + 1), abort_flag, err))) break;
+          if (nxt.live0) { issue_s(0, kslot(j + 1)); tc_commit(bar(B_S + 0)); }
+        }
+        if (cur.live1) {
+          if (!(ok = mbar_wait(bar(B_P + 1), pc[1] & 1u, abort_flag, err))) break;
+          ++pc[1];
+          tc_fence_after();
+          issue_pv(1, vslot(j), acc[1]);
+          acc[1] = true;
+        }
+        tc_commit(bar(B_EMPTY + vslot(j)));
+        if (hn) {
+          if (nxt.live1) { issue_s(1, kslot(j + 1)); tc_commit(bar(B_S + 1)); }
+          tc_commit(bar(B_EMPTY + kslot(j + 1)));
+        }
+        cur = nxt;
+        have = hn;
+        ++j;
+      }
+      tc_commit(bar(B_O + 0));
+      tc_commit(bar(B_O + 1));
+      // Wait for every MMA issued here before TMEM and shared memory go away.
+      tc_commit(bar(B_DRAIN));
+      mbar_wait(bar(B_DRAIN), 0, abort_flag, nullptr, 1000000000ull);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax
+    const int t = (warp - 4) >> 2;
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_base + C::col_s(t);
+    const uint32_t tO = tmem + lane_base + C::col_o(t);
+    const int grow = t * 128 + row;
+    const bool rvalid = grow < it.q_valid;
+    const int qpos = it.q_pos0 + grow;
+    const bool varlen = plan.n_docs > 0;
+    const int row_lo = rvalid ? (varlen ? doc_start(plan.cu_seqlens, plan.n_docs, qpos) : kLoNone) : kHiNone;
+    const int row_hi = rvalid ? (plan.causal ? qpos : kHiNone) : kLoNone;
+    const float scale_log2 = plan.scale_log2;
+    const int full_lo = t == 0 ? it.full_lo[0] : it.full_lo[1];
+    const int full_hi = t == 0 ? it.full_hi[0] : it.full_hi[1];
+
+    float m_used = -CUDART_INF_F;
+    float l = 0.f;
+    uint32_t n_tiles = 0;
+    bool ok = true;
+    KIter ki;
+    make_iter(it, ki);
+    KTile kt;
+    while (ki.next(kt)) {
+      if (!(t == 0 ? kt.live0 : kt.live1)) continue;
+      ok = mbar_wait(bar(B_S + t), n_tiles & 1u, abort_flag, err);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t s[128];
+      tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+      tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+      tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
+      tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
+      tc_wait_ld();
+      const bool full = kt.valid == CP_KV_TILE && kt.pos >= full_lo && kt.pos + CP_KV_TILE - 1 <= full_hi;
+      if (!full) {
+        const int clo = row_lo - kt.pos;
+        const int chi = min(row_hi - kt.pos, kt.valid - 1);
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c < clo || c > chi) s[c] = __float_as_uint(-CUDART_INF_F);
+      }
+      float mx0 = -CUDART_INF_F, mx1 = -CUDART_INF_F, mx2 = -CUDART_INF_F, mx3 = -CUDART_INF_F;
+#pragma unroll
+      for (int c = 0; c < 128; c += 4) {
+        mx0 = fmaxf(mx0, __uint_as_float(s[c + 0]));
+        mx1 = fmaxf(mx1, __uint_as_float(s[c + 1]));
+        mx2 = fmaxf(mx2, __uint_as_float(s[c + 2]));
+        mx3 = fmaxf(mx3, __uint_as_float(s[c + 3]));
+      }
+      const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * scale_log2;
+      const bool need = m_tile > m_used + 8.0f;
+      float alpha = 1.f;
+      if (need) {
+        alpha = ex2_approx(m_used - m_tile);
+        m_used = m_tile;
+        l *= alpha;
+      }
+      const float neg_ref = (m_used == -CUDART_INF_F) ? 0.f : -m_used;
+      float ls0 = 0.f, ls1 = 0.f;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const float p0 = ex2_approx(fmaf(__uint_as_float(s[half * 64 + 2 * c]), scale_log2, neg_ref));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(s[half * 64 + 2 * c + 1]), scale_log2, neg_ref));
+          ls0 += p0;
+          ls1 += p1;
+          pk[c] = pack_bf16x2(p0, p1);
+        }
+        tmem_st32(tS + half * 32, pk);
+      }
+      l += ls0 + ls1;
+      if (n_tiles > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll 1
+        for (int ch = 0; ch < DH / 32; ++ch) {
+          uint32_t o[32];
+          tmem_ld32(tO + ch * 32, o);
+          tc_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(tO + ch * 32, o);
+        }
+      }
+      tc_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(B_P + t));
+      ++n_tiles;
+    }
+    if (ok) {
+      ok = mbar_wait(bar(B_O + t), 0, abort_flag, err);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    if (ok) {
+      tc_fence_after();
+      const cp_pair_desc* pd = it.pd;
+      const int orow = it.out_row0 + grow;
+      float* op = pd->o + ((size_t)orow * plan.hq + it.h) * DH;
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      if (n_tiles > 0) {
+#pragma unroll 1
+        for (int ch = 0; ch < DH / 32; ++ch) {
+          uint32_t o[32];
+          tmem_ld32(tO + ch * 32, o);
+          tc_wait_ld();
+          if (rvalid) {
+            float4* dst = reinterpret_cast<float4*>(op + ch * 32);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              float4 v;
+              v.x = l > 0.f ? __uint_as_float(o[4 * i + 0]) * inv_l : 0.f;
+              v.y = l > 0.f ? __uint_as_float(o[4 * i + 1]) * inv_l : 0.f;
+              v.z = l > 0.f ? __uint_as_float(o[4 * i + 2]) * inv_l : 0.f;
+              v.w = l > 0.f ? __uint_as_float(o[4 * i + 3]) * inv_l : 0.f;
+              dst[i] = v;
+            }
+          }
+        }
+      } else if (rvalid) {
+        float4* dst = reinterpret_cast<float4*>(op);
+        for (int i = 0; i < DH / 4; ++i) dst[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      if (rvalid) {
+        const float lse = l > 0.f ? (m_used + __log2f(l)) * 0.69314718055994531f : -CUDART_INF_F;
+        pd->lse[(size_t)it.h * pd->lse_ld + orow] = lse;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+template <int DH>
+static cudaError_t launch_attn_dh(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                  const cp_attn_plan& plan, cudaStream_t stream) {
+  using C = AttnCfg<DH>;
+  static bool configured = false;  // per process; attribute is per function
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  if (plan.total_ctas <= 0) return cudaSuccess;
+  attn_fwd_kernel<DH><<<plan.total_ctas, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, plan);
+  launch_counter()++;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn(int dh, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                        const cp_attn_plan& plan, cudaStream_t stream) {
+  if (dh == 128) return launch_attn_dh<128>(tq, tk, tv, plan, stream);
+  return launch_attn_dh<64>(tq, tk, tv, plan, stream);
+}
+
+cudaError_t attn_err_word(uint32_t** dev_ptr) {
+  return cudaGetSymbolAddress(reinterpret_cast<void**>(dev_ptr), g_attn_err);
+}
+
+}  // namespace cp

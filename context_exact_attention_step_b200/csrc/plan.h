@@ -1,0 +1,79 @@
+// Launch plans shared by the host scheduler and the sm_100a kernels.
+//
+// A plan is a small POD passed by value as a __grid_constant__ kernel
+// parameter, so every launch is self-describing (no host->device copy of a
+// work list, nothing to allocate, capturable in a CUDA graph).
+#pragma once
+#include <stdint.h>
+
+#define CP_MAX_SEGS 4        // row segments per side of one block pair
+#define CP_MAX_PAIRS 48      // block pairs per attention launch
+#define CP_MAX_TASKS 32      // merge tasks per merge launch
+#define CP_MAX_INPUTS 192    // merge inputs per merge launch
+#define CP_Q_TILE 256        // query rows per CTA (two 128-row MMA tiles)
+#define CP_KV_TILE 128       // key/value rows per pipeline stage
+
+// A run of consecutive buffer rows whose global token positions are also
+// consecutive.  buf_row: first row in the Q/K/V buffer; pos: global position
+// of that row; len: number of rows; out_row: first row in the output buffer
+// (Q side only).
+struct cp_seg {
+  int32_t buf_row;
+  int32_t pos;
+  int32_t len;
+  int32_t out_row;
+};
+
+// One block pair of a ring step: some query rows of rank r against the
+// key/value rows of shard j.
+struct cp_pair_desc {
+  int32_t nq, nk;
+  cp_seg q[CP_MAX_SEGS];
+  cp_seg k[CP_MAX_SEGS];
+  int32_t qtiles;     // sum over q segments of ceil(len / CP_Q_TILE)
+  int32_t cta_begin;  // first CTA of this pair in the launch
+  int32_t reverse;    // visit the query tiles last-first (heaviest first under causal)
+  int32_t lse_ld;     // row pitch of the LSE output ([hq][lse_ld])
+  float* o;           // O output, [rows][hq][dh] fp32
+  float* lse;         // LSE output, [hq][lse_ld] fp32
+};
+
+struct cp_attn_plan {
+  int32_t n_pairs;
+  int32_t total_ctas;
+  int32_t hq, hkv;
+  int32_t causal;
+  int32_t n_docs;               // 0: no document mask
+  const int32_t* cu_seqlens;    // device, n_docs + 1 entries
+  float scale_log2;             // softmax_scale * log2(e)
+  uint32_t* err;                // device error word (bounded-wait timeouts)
+  cp_pair_desc pairs[CP_MAX_PAIRS];
+};
+
+// Merge: rows [out_row0, out_row0 + rows) of the output are the LSE-weighted
+// fold of n_in partial results; input i supplies row (row0 + x) for output
+// row (out_row0 + x).
+struct cp_merge_input {
+  const float* o;      // [.][h][dh]
+  const float* lse;    // [h][lse_ld]
+  int32_t row0;
+  int32_t lse_ld;
+};
+
+struct cp_merge_task {
+  int32_t out_row0;
+  int32_t rows;
+  int32_t n_in;
+  int32_t in_begin;
+};
+
+struct cp_merge_plan {
+  int32_t n_tasks;
+  int32_t h, dh;
+  int32_t lse_out_ld;
+  float* o_out;          // [.][h][dh]
+  float* lse_out;        // [h][lse_out_ld]
+  uint16_t* o_out_bf16;  // optional bf16 copy of O (nullable)
+  cp_merge_task tasks[CP_MAX_TASKS];
+  cp_merge_input inputs[CP_MAX_INPUTS];
+};

@@ -1,0 +1,242 @@
+/*
+ * cp_attn.h -- C ABI of the B200 (sm_100a) context-parallel exact attention
+ * library: ring-step block attention producing partial (O, LSE), the fp32 LSE
+ * merge, the zigzag reorder and the Ulysses sequence<->head transpose, with
+ * the P ranks of a context-parallel group held as virtual ranks on one GPU.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Tensor arguments are DEVICE pointers owned by the caller (allocate them
+ *    however you like, e.g. through PyTorch).  The library allocates no device
+ *    memory; calls that need scratch space take a caller workspace.
+ *  - Host arrays (chunk lists, pointer lists, cu_seqlens_host) are read during
+ *    the call only and may be freed when it returns.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *    NULL = legacy default stream) and returns before the GPU work finishes.
+ *  - Layouts are row-major, token-major: a Q/K/V/O tensor is [rows][heads][dh]
+ *    (the pages' [batch, seq_len, heads, head_dim] with batch = 1 and no
+ *    padding between heads), an LSE tensor is [heads][rows].
+ *  - Every device pointer must be 16-byte aligned, and row pitches follow from
+ *    the shapes (no strides).
+ *  - Errors: every call returns a cp_status.  Arguments are validated before
+ *    anything is launched; on error nothing is launched, nothing is written,
+ *    and cp_last_error_string() (thread-local) describes the problem.  The
+ *    library never aborts the process and never prints.
+ *  - Kernels that wait on hardware barriers give up after a bounded time and
+ *    record it in a device error word read by cp_device_error(); they never
+ *    trap.
+ */
+#ifndef CP_ATTN_H
+#define CP_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  CP_OK = 0,
+  CP_ERR_INVALID_ARG = 1,  /* a size, count or pointer is out of range       */
+  CP_ERR_UNSUPPORTED = 2,  /* valid request outside what this build supports  */
+  CP_ERR_ALIGNMENT = 3,    /* a device pointer is not 16-byte aligned        */
+  CP_ERR_WORKSPACE = 4,    /* workspace missing or smaller than required      */
+  CP_ERR_CUDA = 5          /* the CUDA runtime reported an error              */
+} cp_status;
+
+typedef enum { CP_BF16 = 0, CP_FP32 = 1 } cp_dtype;
+typedef enum { CP_MASK_NONE = 0, CP_MASK_CAUSAL = 1 } cp_mask;
+typedef enum { CP_LAYOUT_CONTIGUOUS = 0, CP_LAYOUT_ZIGZAG = 1 } cp_layout;
+typedef enum { CP_SEQ_TO_HEAD = 0, CP_HEAD_TO_SEQ = 1 } cp_dir;
+
+/* A run of consecutive rows of a Q or K/V buffer whose global token
+ * positions are consecutive: rows [row, row + len) of the buffer (in list
+ * order) hold positions [start, start + len). */
+typedef struct {
+  int32_t start;
+  int32_t len;
+} cp_chunk;
+
+#define CP_MAX_CHUNKS 4
+
+/* Description of the last error returned on the calling thread. */
+const char* cp_last_error_string(void);
+
+/* Library version string. */
+const char* cp_version(void);
+
+/*
+ * cp_block_attn_fwd -- one ring step for one virtual rank: the rank's query
+ * shard against one key/value block, with that block pair's mask offsets.
+ *
+ * Computes, for every query row i and query head h (kv head g = h / (hq/hkv)),
+ *   s_j = softmax_scale * q_i . k_j over the admitted keys j,
+ *   O_i = sum_j softmax(s)_j v_j  (normalised within this block pair),
+ *   LSE_i = ln sum_j exp(s_j)     (natural log of the scaled scores),
+ * where key j is admitted iff (mask == CP_MASK_CAUSAL ? pos(j) <= pos(i) : 1)
+ * and (n_docs > 0 ? doc(pos(i)) == doc(pos(j)) : 1).  Rows with no admitted
+ * key get O = 0 and LSE = -inf.  This is the block step of Ring Attention
+ * ("序列並行（Sequence Parallelism）" concept page (compassingai), "Ring
+ * Attention 的不同思路" steps 1-4 and 技術原理 §二, S = Q K^T / sqrt(d_k)),
+ * with the per-block mask offsets of the "Context Parallelism" write-up
+ * (pwwt.cn) §3.3, and packed documents through cu_seqlens (XTuner tutorial
+ * ch09 §9.5).
+ *
+ *   q            [n_q][hq][dh] bf16 (dtype must be CP_BF16)
+ *   k, v         [n_k][hkv][dh] bf16
+ *   q_chunks     host, nq_chunks (1..CP_MAX_CHUNKS) entries covering the n_q
+ *                rows in order; positions of the query rows
+ *   k_chunks     host, nk_chunks entries covering the n_k rows; key positions
+ *   mask         CP_MASK_NONE or CP_MASK_CAUSAL (by global position)
+ *   cu_seqlens_dev  device int32 [n_docs + 1], 0 = first, strictly increasing
+ *                (document lengths > 0), covering every position used; NULL
+ *                with n_docs = 0 for no document mask
+ *   softmax_scale  > 0, or <= 0 for 1/sqrt(dh)
+ *   o            out, [n_q][hq][dh] fp32
+ *   lse          out, [hq][n_q] fp32
+ * Supported: dh in {64, 128}; hq % hkv == 0; 1 <= n_q, n_k < 2^30.
+ */
+cp_status cp_block_attn_fwd(const void* q, const void* k, const void* v, cp_dtype dtype, int n_q, int n_k,
+                            int hq, int hkv, int dh, const cp_chunk* q_chunks, int nq_chunks,
+                            const cp_chunk* k_chunks, int nk_chunks, cp_mask mask,
+                            const int32_t* cu_seqlens_dev, int n_docs, float softmax_scale, float* o,
+                            float* lse, void* stream);
+
+/*
+ * cp_lse_merge -- fold n_parts partial results over the same rows:
+ *   LSE = ln sum_i exp(LSE_i),  O = sum_i exp(LSE_i - LSE) * O_i,
+ * in fp32; partials with LSE_i = -inf for a row contribute nothing there (their
+ * O is not read); rows where every LSE_i is -inf get O = 0, LSE = -inf.  The
+ * block-granular form of the online-softmax recurrence ("序列並行" concept page
+ * (compassingai), 技術原理 §二).
+ *
+ *   o_parts      host array of n_parts device pointers, each [rows][h][dh] fp32
+ *   lse_parts    host array of n_parts device pointers, each [h][rows] fp32
+ *   o_out        out, [rows][h][dh] fp32 (may not alias an input)
+ *   lse_out      out, [h][rows] fp32
+ *   o_out_bf16   optional out, [rows][h][dh] bf16 copy of O (NULL to skip)
+ * Supported: 1 <= n_parts <= 64, dh in {64, 128}.
+ */
+cp_status cp_lse_merge(int n_parts, const float* const* o_parts, const float* const* lse_parts, int rows, int h,
+                       int dh, float* o_out, float* lse_out, void* o_out_bf16, void* stream);
+
+/*
+ * cp_ring_attn_workspace_size -- bytes of workspace cp_ring_attn_fwd needs for
+ * these arguments (partials of every live block pair, plus bf16 copies of Q,
+ * K, V when dtype is CP_FP32).  cu_seqlens_host may be NULL; when given, the
+ * same array must be passed to cp_ring_attn_fwd.
+ */
+cp_status cp_ring_attn_workspace_size(int S, int hq, int hkv, int dh, int P, cp_layout layout, cp_mask mask,
+                                      cp_dtype dtype, const int32_t* cu_seqlens_host, int n_docs, size_t* bytes);
+
+/*
+ * cp_ring_attn_fwd -- exact attention of a whole sequence split over P
+ * virtual ranks, computed as Ring Attention does it: rank r keeps its query
+ * shard, at step t = 0..P-1 it holds key/value shard j = (r - t) mod P, every
+ * live block pair yields a partial (O, LSE) (cp_block_attn_fwd semantics) and
+ * the partials of each rank are folded by the LSE merge.  Block pairs the mask
+ * leaves empty are skipped, as are the query rows of a pair that see none of
+ * its keys.  ("序列並行" concept page (compassingai), Ring Attention steps 1-4;
+ * "Context Parallelism" write-up (pwwt.cn) §2.2, §3.3; zigzag balancing:
+ * "长上下文序列并行训练深度解析" (mooersco) timeline, Striped / zigzag.)
+ *
+ *   q            [S][hq][dh], k, v [S][hkv][dh], bf16 or fp32 (fp32 inputs are
+ *                rounded to bf16, nearest-even, before use) ALREADY in the
+ *                rank-major sharded order of `layout`: rank r holds rows
+ *                [r*S/P, (r+1)*S/P).  CP_LAYOUT_CONTIGUOUS: rank r holds
+ *                positions [r*S/P, (r+1)*S/P).  CP_LAYOUT_ZIGZAG: rank r holds
+ *                chunk r then chunk 2P-1-r of the 2P chunks of S/(2P) tokens
+ *                (cp_zigzag_reorder produces this order).
+ *   cu_seqlens_host, cu_seqlens_dev  the same document table on host and device
+ *                (n_docs + 1 entries; both NULL and n_docs = 0 for none); the
+ *                host copy lets the scheduler skip pairs across documents
+ *   o            out, [S][hq][dh] fp32, in the same sharded order as q
+ *   lse          out, [hq][S] fp32, same order
+ *   workspace    device scratch of at least cp_ring_attn_workspace_size bytes,
+ *                256-byte aligned; its contents are overwritten
+ * Supported: 1 <= P <= 16, S % P == 0 (S % 2P == 0 for zigzag), dh in {64,128},
+ * hq % hkv == 0.
+ */
+cp_status cp_ring_attn_fwd(const void* q, const void* k, const void* v, cp_dtype dtype, int S, int hq, int hkv,
+                           int dh, int P, cp_layout layout, cp_mask mask, const int32_t* cu_seqlens_host,
+                           const int32_t* cu_seqlens_dev, int n_docs, float softmax_scale, float* o, float* lse,
+                           void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * cp_ulysses_permute -- the DeepSpeed-Ulysses all-to-all transpose as a local
+ * permute ("序列並行" concept page (compassingai), 技術原理 §三 "Ulysses 的
+ * AllToAll 轉置"; "Context Parallelism" write-up (pwwt.cn) §2.3), with n = S/P:
+ *   CP_SEQ_TO_HEAD: in [P][n][h][dh] -> out [P][S][h/P][dh],
+ *                   out[r][p*n + s][h'] = in[p][s][r*h/P + h']
+ *   CP_HEAD_TO_SEQ: the inverse.
+ * Bit-exact copy of elem_bytes-sized elements (2 for bf16, 4 for fp32).
+ * For GQA call it on Q with h = hq and on K, V with h = hkv.
+ * Supported: P | S, P | h; in and out must not overlap.
+ */
+cp_status cp_ulysses_permute(const void* in, void* out, int P, int S, int h, int dh, int elem_bytes, cp_dir dir,
+                             void* stream);
+
+/*
+ * cp_zigzag_reorder -- natural token order <-> rank-major zigzag order
+ * (rank i holds chunks i and 2P-1-i of 2P chunks of S/(2P) rows).  in/out are
+ * [batch][S][row_bytes] byte arrays: use batch = 1, row_bytes = h*dh*elem for
+ * Q/K/V/O, and batch = h, row_bytes = 4 for an fp32 LSE [h][S].
+ * inverse = 0: natural -> zigzag; 1: zigzag -> natural.  Bit-exact.
+ * Supported: S % (2P) == 0; in and out must not overlap.
+ */
+cp_status cp_zigzag_reorder(const void* in, void* out, int P, int S, int batch, int row_bytes, int inverse,
+                            void* stream);
+
+/*
+ * cp_ulysses_attn_workspace_size / cp_ulysses_attn_fwd -- the Ulysses path:
+ * seq->head transpose of Q (hq heads) and K, V (hkv heads), local attention of
+ * every head group over the whole sequence (P = 1 ring, GQA inside the group),
+ * head->seq transpose of O back.  Inputs q [P][S/P][hq][dh], k, v
+ * [P][S/P][hkv][dh] bf16 (sequence-sharded, natural position order); outputs o
+ * [P][S/P][hq][dh] fp32 and lse [hq][S] fp32 (natural positions).
+ * Supported: P | hkv (the Ulysses head limit; KV heads are not replicated),
+ * P | S, dh in {64, 128}.
+ */
+cp_status cp_ulysses_attn_workspace_size(int S, int hq, int hkv, int dh, int P, size_t* bytes);
+cp_status cp_ulysses_attn_fwd(const void* q, const void* k, const void* v, int S, int hq, int hkv, int dh, int P,
+                              cp_mask mask, float softmax_scale, float* o, float* lse, void* workspace,
+                              size_t ws_bytes, void* stream);
+
+/*
+ * Host-only inspection of the ring-step schedule (no GPU needed).  For every
+ * rank r and step t (index r*P + t):
+ *   src[r*P+t]        the key/value shard j = (r - t) mod P held at that step
+ *   launched[r*P+t]   1 if the block pair is computed, 0 if skipped as empty
+ *   q_rows[r*P+t]     query rows of the pair that are computed
+ *   live_pairs[r*P+t] number of admitted (query, key) pairs in the block pair
+ * Any output pointer may be NULL.  cu_seqlens_host as in cp_ring_attn_fwd.
+ */
+cp_status cp_ring_schedule(int S, int P, cp_layout layout, cp_mask mask, const int32_t* cu_seqlens_host,
+                           int n_docs, int32_t* src, int32_t* launched, int32_t* q_rows, int64_t* live_pairs);
+
+/* Number of admitted (query, key) pairs of the whole sequence: the unit of
+ * the causal-effective FLOP count 4 * dh * hq * pairs.  Host only. */
+cp_status cp_count_live_pairs(int S, cp_mask mask, const int32_t* cu_seqlens_host, int n_docs, int64_t* pairs);
+
+/* Reads (and, if clear != 0, resets) the device error word of the current
+ * device: 0 = no kernel gave up waiting; bit 0 = a bounded wait timed out.
+ * Synchronous. */
+cp_status cp_device_error(uint32_t* bits, int clear);
+
+/* Total number of kernels this library has launched in the process (all
+ * devices, all threads).  Host only. */
+cp_status cp_kernel_launch_count(uint64_t* count);
+
+/* Profiling hook: when non-NULL, the composite calls (cp_ring_attn_fwd,
+ * cp_ulysses_attn_fwd) made afterwards on the calling thread record
+ * `attn_begin` / `attn_end` (cudaEvent_t passed as void*) on their stream
+ * immediately before their first and after their last block-attention launch,
+ * and `merge_end` after their last merge launch.  Pass NULLs to turn it off. */
+cp_status cp_set_profile_events(void* attn_begin, void* attn_end, void* merge_end);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CP_ATTN_H */

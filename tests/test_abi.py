@@ -1,0 +1,153 @@
+"""CPU checks of the C ABI: the library loads, exports every entry point the
+header declares, validates arguments before launching anything, and its host
+ring-step scheduler agrees with the oracle's brute-force mask counts."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from context_exact_attention_step_b200 import _lib, api
+from context_exact_attention_step_b200._lib import cp_chunk, lib
+from oracle import ref
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from context_exact_attention_step_b200 import build
+    build.build()
+
+
+def header_functions():
+    with open(os.path.join(ROOT, "include", "cp_attn.h")) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"^\s*(?:const char\*|cp_status)\s+(cp_\w+)\s*\(", text, re.M)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = header_functions()
+    assert len(names) >= 13
+    L = lib()
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(_lib.EXPORTS)
+    assert b"sm_100a" in L.cp_version()
+
+
+FAKE = ctypes.c_void_p(1 << 20)        # aligned, never dereferenced on error paths
+MISALIGNED = ctypes.c_void_p((1 << 20) + 8)
+
+
+def _block(q=FAKE, k=FAKE, v=FAKE, dtype=_lib.CP_BF16, n_q=256, n_k=256, hq=4, hkv=4, dh=128, nqc=1, nkc=1,
+           mask=_lib.CP_MASK_CAUSAL, cu=None, n_docs=0, o=FAKE, lse=FAKE, qchunks=None):
+    qc = qchunks or (cp_chunk * 1)(cp_chunk(0, n_q))
+    kc = (cp_chunk * 1)(cp_chunk(0, n_k))
+    return lib().cp_block_attn_fwd(q, k, v, dtype, n_q, n_k, hq, hkv, dh, qc, nqc, kc, nkc, mask,
+                                   cu or ctypes.c_void_p(0), n_docs, 0.0, o, lse, ctypes.c_void_p(0))
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dh=96), _lib.CP_ERR_UNSUPPORTED),
+    (dict(hq=6, hkv=4), _lib.CP_ERR_INVALID_ARG),
+    (dict(dtype=_lib.CP_FP32), _lib.CP_ERR_UNSUPPORTED),
+    (dict(q=ctypes.c_void_p(0)), _lib.CP_ERR_INVALID_ARG),
+    (dict(k=MISALIGNED), _lib.CP_ERR_ALIGNMENT),
+    (dict(o=MISALIGNED), _lib.CP_ERR_ALIGNMENT),
+    (dict(n_q=0), _lib.CP_ERR_INVALID_ARG),
+    (dict(nqc=5), _lib.CP_ERR_UNSUPPORTED),
+    (dict(n_docs=3), _lib.CP_ERR_INVALID_ARG),
+    (dict(mask=7), _lib.CP_ERR_INVALID_ARG),
+    (dict(qchunks=(cp_chunk * 1)(cp_chunk(0, 100))), _lib.CP_ERR_INVALID_ARG),
+])
+def test_block_attn_rejects_bad_arguments(kw, status):
+    assert _block(**kw) == status
+    assert len(lib().cp_last_error_string()) > 0
+
+
+def _ring(S=1024, hq=4, hkv=4, dh=64, P=4, layout=_lib.CP_LAYOUT_CONTIGUOUS, cu=None, n_docs=0, ws=FAKE, wsb=1 << 40,
+          o=FAKE):
+    return lib().cp_ring_attn_fwd(FAKE, FAKE, FAKE, _lib.CP_BF16, S, hq, hkv, dh, P, layout, _lib.CP_MASK_CAUSAL,
+                                  cu, ctypes.c_void_p(0) if not n_docs else FAKE, n_docs, 0.0, o, FAKE, ws, wsb,
+                                  ctypes.c_void_p(0))
+
+
+def test_ring_rejects_bad_arguments():
+    assert _ring(S=1000, P=3) == _lib.CP_ERR_INVALID_ARG            # P does not divide S
+    assert _ring(S=1028, P=4, layout=_lib.CP_LAYOUT_ZIGZAG) == _lib.CP_ERR_INVALID_ARG  # 2P does not divide S
+    assert _ring(P=17) == _lib.CP_ERR_UNSUPPORTED
+    assert _ring(ws=ctypes.c_void_p(0), wsb=0) == _lib.CP_ERR_WORKSPACE
+    assert _ring(wsb=16) == _lib.CP_ERR_WORKSPACE
+    assert _ring(o=MISALIGNED) == _lib.CP_ERR_ALIGNMENT
+    bad = (ctypes.c_int32 * 3)(0, 600, 500)
+    assert _ring(cu=bad, n_docs=2) == _lib.CP_ERR_INVALID_ARG       # not increasing
+    short = (ctypes.c_int32 * 3)(0, 600, 1000)
+    assert _ring(cu=short, n_docs=2) == _lib.CP_ERR_INVALID_ARG     # does not end at S
+
+
+def test_permute_and_merge_reject_bad_arguments():
+    L = lib()
+    # Ulysses head limit: P must divide the head count
+    assert L.cp_ulysses_permute(FAKE, ctypes.c_void_p(1 << 30), 8, 1024, 4, 128, 2, 0, None) == _lib.CP_ERR_UNSUPPORTED
+    assert L.cp_ulysses_permute(FAKE, ctypes.c_void_p(1 << 30), 4, 1022, 8, 128, 2, 0, None) == _lib.CP_ERR_INVALID_ARG
+    assert L.cp_ulysses_permute(FAKE, FAKE, 4, 1024, 8, 128, 2, 0, None) == _lib.CP_ERR_INVALID_ARG  # overlap
+    assert L.cp_zigzag_reorder(FAKE, ctypes.c_void_p(1 << 30), 4, 1020, 1, 16, 0, None) == _lib.CP_ERR_INVALID_ARG
+    sz = ctypes.c_size_t(0)
+    assert L.cp_ulysses_attn_workspace_size(1024, 32, 4, 128, 8, ctypes.byref(sz)) == _lib.CP_ERR_UNSUPPORTED
+    parts = (ctypes.c_void_p * 1)(1 << 20)
+    assert L.cp_lse_merge(0, parts, parts, 16, 2, 128, FAKE, FAKE, None, None) == _lib.CP_ERR_UNSUPPORTED
+    assert L.cp_lse_merge(1, parts, parts, 16, 2, 96, FAKE, FAKE, None, None) == _lib.CP_ERR_UNSUPPORTED
+    assert L.cp_lse_merge(1, parts, parts, 16, 2, 128, FAKE, FAKE, None, None) == _lib.CP_ERR_INVALID_ARG  # alias
+
+
+# ------------------------------------------------------------ scheduler
+@pytest.mark.parametrize("layout", ["contiguous", "zigzag"])
+@pytest.mark.parametrize("P", [1, 2, 4, 8])
+@pytest.mark.parametrize("causal", [True, False])
+def test_schedule_matches_bruteforce(layout, P, causal):
+    S = 16 * P * 2
+    sch = api.ring_schedule(S, P, layout, causal)
+    cls = ref.pair_classes(S, P, layout, causal)
+    for r in range(P):
+        for t in range(P):
+            j, live, tot = cls[(r, t)]
+            i = r * P + t
+            assert sch["src"][i] == j
+            assert sch["live_pairs"][i] == live
+            assert sch["launched"][i] == (1 if live > 0 else 0)
+
+
+def test_schedule_varlen_matches_bruteforce():
+    S, P = 256, 4
+    cu = [0, 3, 70, 71, 200, 256]
+    sch = api.ring_schedule(S, P, "zigzag", True, cu)
+    cls = ref.pair_classes(S, P, "zigzag", True, cu)
+    for (r, t), (j, live, _) in cls.items():
+        assert sch["live_pairs"][r * P + t] == live
+        assert sch["launched"][r * P + t] == (1 if live else 0)
+        if live:
+            # every query row that admits a key of the pair is computed
+            qp = ref.shard_positions(S, P, "zigzag", r)
+            kp = ref.shard_positions(S, P, "zigzag", j)
+            rows_live = ref.explicit_mask(qp, kp, True, cu).any(axis=1).sum()
+            assert sch["q_rows"][r * P + t] >= rows_live
+
+
+def test_schedule_skip_counts_for_the_workloads():
+    # contiguous causal P=4: P(P+1)/2 live pairs; zigzag P=8: all P^2 live
+    assert api.ring_schedule(32768, 4, "contiguous")["launched"].sum() == 10
+    z = api.ring_schedule(65536, 8, "zigzag")
+    assert z["launched"].sum() == 64
+    c = 65536 // 16
+    # off-diagonal zigzag pairs compute half the query rows (or all rows vs half the keys)
+    assert set(np.unique(z["live_pairs"])) == {2 * c * c, 2 * c * c + c}
+
+
+def test_live_pair_count_against_oracle():
+    cu = [0, 5, 6, 40, 64]
+    assert api.count_live_pairs(64, True, cu) == ref.live_pair_count(64, True, cu)
+    assert api.count_live_pairs(64, True) == 64 * 65 // 2
+    assert api.count_live_pairs(64, False) == 64 * 64
+    assert api.count_live_pairs(131072, True) == 131072 * 131073 // 2

@@ -1,0 +1,74 @@
+"""GPU parity of the layout kernels: bit-exact against the oracle's numpy
+index formulas (Ulysses transpose, zigzag reorder), through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+from context_exact_attention_step_b200 import api, synth
+from oracle import ref
+
+pytestmark = pytest.mark.gpu
+
+
+def bits(t: torch.Tensor) -> np.ndarray:
+    t = t.detach().cpu()
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).numpy()
+    return t.view(torch.int32).numpy() if t.element_size() == 4 else t.numpy()
+
+
+@pytest.mark.parametrize("P,S,h,dh,dtype", [
+    (4, 64, 8, 128, torch.bfloat16),
+    (8, 1024, 32, 128, torch.bfloat16),
+    (8, 1024, 8, 128, torch.bfloat16),      # GQA K/V: one head per rank
+    (2, 96, 4, 64, torch.float32),
+    (4, 40, 4, 3, torch.bfloat16),          # odd row size: narrow copy units
+    (1, 32, 4, 16, torch.bfloat16),         # P = 1 is the identity
+])
+def test_ulysses_permute_bit_exact(P, S, h, dh, dtype):
+    x = synth.normal((S, h, dh), 11, 1.0, dtype).cuda()
+    y = api.ulysses_permute(x, P, "seq_to_head")
+    want = ref.ulysses_seq_to_head(bits(x).reshape(P, S // P, h, dh), P)
+    assert np.array_equal(bits(y), want)
+    back = api.ulysses_permute(y, P, "head_to_seq")
+    assert np.array_equal(bits(back), bits(x))
+
+
+def test_ulysses_permute_full_size_q():
+    # the 128K-token GQA workload's Q (32 heads) and K (8 heads), P = 8
+    P, S, dh = 8, 131072, 128
+    for h, seed in ((32, 1), (8, 2)):
+        x = synth.normal((S, h, dh), seed, 0.5, torch.bfloat16).cuda()
+        y = api.ulysses_permute(x, P, "seq_to_head")
+        # spot-check whole rows of every (r, p) block against the formula
+        xb = x.view(P, S // P, h, dh)
+        for r in range(P):
+            for p in range(P):
+                for s in (0, 1, S // P - 1, 777 % (S // P)):
+                    got = y[r, p * (S // P) + s]
+                    exp = xb[p, s, r * (h // P):(r + 1) * (h // P)]
+                    assert torch.equal(got.view(torch.int16), exp.view(torch.int16))
+        back = api.ulysses_permute(y, P, "head_to_seq")
+        assert torch.equal(back.view(torch.int16), x.view(torch.int16))
+
+
+@pytest.mark.parametrize("P,S,shape,dtype", [
+    (4, 64, (8, 128), torch.bfloat16),
+    (8, 4096, (32, 128), torch.bfloat16),
+    (2, 40, (3,), torch.float32),
+    (3, 36, (2, 5), torch.bfloat16),
+])
+def test_zigzag_bit_exact(P, S, shape, dtype):
+    x = synth.normal((S,) + shape, 5, 1.0, dtype).cuda()
+    y = api.zigzag_reorder(x, P)
+    assert np.array_equal(bits(y), ref.zigzag_reorder(bits(x), P))
+    z = api.zigzag_reorder(y, P, inverse=True)
+    assert np.array_equal(bits(z), bits(x))
+
+
+def test_zigzag_lse_rows():
+    P, S, h = 8, 4096, 32
+    lse = synth.normal((h, S), 9, 1.0, torch.float32).cuda()
+    y = api.zigzag_reorder(lse, P, seq_dim=1)
+    assert np.array_equal(bits(y), ref.zigzag_reorder(bits(lse), P, axis=1))
+    assert torch.equal(api.zigzag_reorder(y, P, inverse=True, seq_dim=1), lse)

@@ -107,13 +107,21 @@ struct KIter {
   }
 };
 
-__device__ __forceinline__ int doc_start(const int32_t* __restrict__ cu, int n_docs, int x) {
+// Index of the document holding position x (cu = prefix sums, n_docs docs).
+__device__ __forceinline__ int doc_index(const int32_t* __restrict__ cu, int n_docs, int x) {
   int lo = 0, hi = n_docs - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
     if (__ldg(cu + mid) <= x) lo = mid; else hi = mid - 1;
   }
-  return __ldg(cu + lo);
+  return lo;
+}
+__device__ __forceinline__ int doc_start(const int32_t* __restrict__ cu, int n_docs, int x) {
+  return __ldg(cu + doc_index(cu, n_docs, x));
+}
+// Last position of the document holding x.
+__device__ __forceinline__ int doc_last(const int32_t* __restrict__ cu, int n_docs, int x) {
+  return __ldg(cu + doc_index(cu, n_docs, x) + 1) - 1;
 }
 
 struct Item {
@@ -155,8 +163,9 @@ __device__ __forceinline__ void decode_item(const cp_attn_plan& plan, Item& it) 
     const bool varlen = plan.n_docs > 0;
     it.vis_lo[t] = varlen ? doc_start(plan.cu_seqlens, plan.n_docs, qa) : kLoNone;
     it.full_lo[t] = varlen ? doc_start(plan.cu_seqlens, plan.n_docs, qb) : kLoNone;
-    it.vis_hi[t] = plan.causal ? qb : kHiNone;
-    it.full_hi[t] = plan.causal ? qa : kHiNone;
+    // upper key limit of a row: itself (causal) or its document's end
+    it.vis_hi[t] = plan.causal ? qb : (varlen ? doc_last(plan.cu_seqlens, plan.n_docs, qb) : kHiNone);
+    it.full_hi[t] = plan.causal ? qa : (varlen ? doc_last(plan.cu_seqlens, plan.n_docs, qa) : kHiNone);
   }
 }
 
@@ -354,7 +363,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int qpos = it.q_pos0 + grow;
     const bool varlen = plan.n_docs > 0;
     const int row_lo = rvalid ? (varlen ? doc_start(plan.cu_seqlens, plan.n_docs, qpos) : kLoNone) : kHiNone;
-    const int row_hi = rvalid ? (plan.causal ? qpos : kHiNone) : kLoNone;
+    const int row_hi =
+        rvalid ? (plan.causal ? qpos : (varlen ? doc_last(plan.cu_seqlens, plan.n_docs, qpos) : kHiNone)) : kLoNone;
     const float scale_log2 = plan.scale_log2;
     const int full_lo = t == 0 ? it.full_lo[0] : it.full_lo[1];
     const int full_hi = t == 0 ? it.full_hi[0] : it.full_hi[1];

@@ -99,7 +99,7 @@ int64_t pair_tile_cost(const std::vector<Seg>& q, const std::vector<Seg>& k, boo
         if (vt <= 0) continue;
         const int qa = qs.pos + off + t * 128, qb = qa + vt - 1;
         const int vis_lo = docs.any() ? docs.start_of(qa) : INT_MIN;
-        const int vis_hi = causal ? qb : INT_MAX;
+        const int vis_hi = causal ? qb : (docs.any() ? docs.end_of(qb) - 1 : INT_MAX);
         for (const Seg& ks : k)
           for (int ko = 0; ko < ks.len; ko += CP_KV_TILE) {
             const int ka = ks.pos + ko, kb = ka + std::min(CP_KV_TILE, ks.len - ko) - 1;

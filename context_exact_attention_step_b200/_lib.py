@@ -24,6 +24,7 @@ EXPORTS = [
     "cp_ring_attn_workspace_size", "cp_ring_attn_fwd", "cp_ulysses_permute", "cp_zigzag_reorder",
     "cp_ulysses_attn_workspace_size", "cp_ulysses_attn_fwd", "cp_ring_schedule", "cp_count_live_pairs",
     "cp_device_error", "cp_kernel_launch_count", "cp_set_profile_events",
+    "cp_ring_attn_fwd_noalloc",
 ]
 
 
@@ -67,6 +68,9 @@ def lib():
     L.cp_ring_attn_fwd.restype = i32
     L.cp_ring_attn_fwd.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, P32, vp, i32, f32, vp, vp,
                                    vp, ctypes.c_size_t, vp]
+    L.cp_ring_attn_fwd_noalloc.restype = i32
+    L.cp_ring_attn_fwd_noalloc.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, P32, vp, i32, f32,
+                                           vp, vp, vp]
     L.cp_ulysses_permute.restype = i32
     L.cp_ulysses_permute.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, vp]
     L.cp_zigzag_reorder.restype = i32

@@ -141,6 +141,36 @@ def ring_attn_fwd(q, k, v, P, layout="contiguous", causal=True, cu_seqlens=None,
     return o, lse
 
 
+def ring_attn_fwd_noalloc(q, k, v, P, layout="contiguous", causal=True, cu_seqlens=None, cu_seqlens_dev=None,
+                          softmax_scale=0.0, o=None, lse=None, stream=None):
+    """ring_attn_fwd without a workspace, for callers that may not allocate
+    device memory while they run: the library keeps the partial results in
+    its own fixed scratch array (CP_NOALLOC_SCRATCH_BYTES per device).  Pass
+    preallocated ``o``, ``lse`` and ``cu_seqlens_dev`` to allocate nothing on
+    this path either.  Calls overlapping on the GPU share that scratch and
+    race; the first call on a device must come before any stream capture."""
+    dtype = q.dtype
+    if dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("q must be bf16 or fp32")
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _need_cuda(n, t, dtype)
+    S, hq, dh = q.shape
+    hkv = k.shape[1]
+    cu_p, n_docs, cu_np = _cu_host(cu_seqlens)
+    if n_docs > 0 and cu_seqlens_dev is None:
+        cu_seqlens_dev = torch.from_numpy(cu_np).to(q.device)
+    if o is None:
+        o = torch.empty((S, hq, dh), device=q.device, dtype=torch.float32)
+    if lse is None:
+        lse = torch.empty((hq, S), device=q.device, dtype=torch.float32)
+    check(lib().cp_ring_attn_fwd_noalloc(_vp(q), _vp(k), _vp(v),
+                                         _lib.CP_FP32 if dtype == torch.float32 else _lib.CP_BF16, S, hq, hkv, dh, P,
+                                         _LAYOUTS[layout], _lib.CP_MASK_CAUSAL if causal else _lib.CP_MASK_NONE,
+                                         cu_p, _vp(cu_seqlens_dev), n_docs, float(softmax_scale), _vp(o), _vp(lse),
+                                         _stream(stream)))
+    return o, lse
+
+
 def ulysses_permute(x, P, direction="seq_to_head", out=None, stream=None):
     """seq_to_head: x [S, h, dh] (= [P][S/P][h][dh]) -> [P, S, h/P, dh].
     head_to_seq: x [P, S, h/P, dh] -> [S, h, dh].  Bit-exact copy."""

@@ -32,11 +32,19 @@ cudaError_t launch_f32_to_bf16(const float* in, void* out, size_t n, cudaStream_
 std::atomic<uint64_t>& launch_counter();
 }  // namespace cp
 
+namespace {
+thread_local std::string g_err;
+}  // namespace
+
+namespace cp {
+// Lets other translation units of the library report an error message.
+void set_error_message(const char* msg) { g_err = msg ? msg : ""; }
+}  // namespace cp
+
 using namespace cp;
 
 namespace {
 
-thread_local std::string g_err;
 thread_local cudaEvent_t g_ev_attn_begin = nullptr, g_ev_attn_end = nullptr, g_ev_merge_end = nullptr;
 
 void record(cudaEvent_t ev, cudaStream_t st) {

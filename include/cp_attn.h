@@ -224,6 +224,34 @@ cp_status cp_count_live_pairs(int S, cp_mask mask, const int32_t* cu_seqlens_hos
  * Synchronous. */
 cp_status cp_device_error(uint32_t* bits, int clear);
 
+/*
+ * cp_ring_attn_fwd_noalloc -- cp_ring_attn_fwd for callers that may not
+ * allocate device memory (for example a plugin whose host application owns
+ * the whole device-memory budget and forbids allocation while it runs, or a
+ * latency-critical loop in which an allocation would stall the device).  The
+ * pages have no counterpart: this is a property of the library, not of the
+ * method.
+ *
+ * Same arguments and results as cp_ring_attn_fwd, without the workspace: the
+ * partial results live in a scratch array of CP_NOALLOC_SCRATCH_BYTES bytes
+ * compiled into the library, which every GPU that uses the library keeps
+ * until the process exits.  The call allocates nothing.
+ *  - Problems whose cp_ring_attn_workspace_size exceeds the scratch are
+ *    rejected with CP_ERR_WORKSPACE and a message giving both sizes.
+ *  - The first call on each device looks up the scratch address of that
+ *    device (cudaGetSymbolAddress); make that first call before any stream
+ *    capture begins.
+ *  - All calls share the one scratch array per device and it keeps whatever
+ *    the last call left there.  Calls whose GPU work overlaps in time (on
+ *    different streams, or from different threads) race on it: order them on
+ *    one stream or synchronise between them.
+ */
+#define CP_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+cp_status cp_ring_attn_fwd_noalloc(const void* q, const void* k, const void* v, cp_dtype dtype, int S, int hq,
+                                   int hkv, int dh, int P, cp_layout layout, cp_mask mask,
+                                   const int32_t* cu_seqlens_host, const int32_t* cu_seqlens_dev, int n_docs,
+                                   float softmax_scale, float* o, float* lse, void* stream);
+
 /* Total number of kernels this library has launched in the process (all
  * devices, all threads).  Host only. */
 cp_status cp_kernel_launch_count(uint64_t* count);

@@ -145,9 +145,11 @@ def max_over_ranks(x, ws):
 
 
 # ----------------------------------------------------------------- workloads
-def make_workload(name):
+def make_workload(name, seq_len=None):
     from context_exact_attention_step_b200 import api, synth
     cfg = dict(synth.CONFIGS[name])
+    if seq_len:
+        cfg["S"] = int(seq_len)
     S, hq, hkv, dh, P = cfg["S"], cfg["hq"], cfg["hkv"], cfg["dh"], cfg["P"]
     dtype = torch.float32 if cfg["dtype"] == "fp32" else torch.bfloat16
     q, k, v = synth.qkv(S, hq, hkv, dh, std=cfg["std"], dtype=dtype)
@@ -377,7 +379,7 @@ def run_ours(args, ws, rank, local):
     from context_exact_attention_step_b200 import build as _build
     _build.build()
     pk = peaks()
-    w = make_workload(args.workload)
+    w = make_workload(args.workload, args.seq_len)
     clocks = Clocks(local)
     clocks.start()
     total_ms, attn_ms, merge_ms, launches = time_steps(w, args.steps, args.warmup, ws)
@@ -445,6 +447,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-permute", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--seq-len", type=int, default=None,
+                    help="override the workload's sequence length (smaller cases for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -16,7 +16,7 @@
 #include <string>
 #include <vector>
 
-#include "../../include/cp_attn.h"
+#include "cp_attn.h"
 #include "plan.h"
 #include "scheduler.h"
 

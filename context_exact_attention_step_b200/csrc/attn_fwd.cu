@@ -40,6 +40,15 @@ std::atomic<uint64_t>& launch_counter();
 __device__ uint32_t g_attn_err = 0;
 
 constexpr int kThreads = 384;
+// Every kPolyEvery-th column pair of an unmasked tile takes the software
+// exp2 on the FMA pipe instead of MUFU (0 disables it).  Measured on B200 the
+// softmax is bound by instruction latency rather than MUFU throughput, and
+// the longer instruction stream of the software path made every tested
+// fraction (1/4, 1/3, 1/2) slower, so it is off by default.
+#ifndef CP_POLY_EVERY
+#define CP_POLY_EVERY 0
+#endif
+constexpr int kPolyEvery = CP_POLY_EVERY;
 constexpr int kLoNone = -(1 << 30);
 constexpr int kHiNone = (1 << 30);
 
@@ -192,7 +201,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + C::kStages * C::kTileBytes);
   // barrier indices
   const int B_Q = 0, B_FULL = 1, B_EMPTY = 1 + C::kStages, B_S = 1 + 2 * C::kStages, B_P = B_S + 2,
-            B_O = B_P + 2, B_DRAIN = B_O + 2, B_COUNT = B_DRAIN + 1;
+            B_O = B_P + 4, B_DRAIN = B_O + 2, B_COUNT = B_DRAIN + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + B_COUNT);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   auto bar = [&](int i) { return smem_addr(bars + i); };
@@ -209,7 +218,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar(B_S + t), 1);
-      mbar_init(bar(B_P + t), 128);
+      mbar_init(bar(B_P + 2 * t + 0), 4);  // one arrive per softmax warp
+      mbar_init(bar(B_P + 2 * t + 1), 4);
       mbar_init(bar(B_O + t), 1);
     }
     mbar_init(bar(B_DRAIN), 1);
@@ -233,124 +243,137 @@ __global__ void __launch_bounds__(kThreads, 1)
   Item it;
   decode_item(plan, it);
 
+  // Registers: launched at 168 per thread (384 threads); inside its own
+  // branch the control warpgroup (warps 0-3) drops to 56 and the two softmax
+  // warpgroups rise to 216: 128 * 56 + 256 * 216 = 62464 <= 384 * 168 = 64512.
+  if (warp < 4) {
+    regs_dec<56>();
+
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      mbar_arrive_expect_tx(bar(B_Q), C::kQBytes);
-      for (int t = 0; t < 2; ++t)
+    // The whole warp runs the loop; one elected lane issues each copy.
+    mbar_arrive_expect_tx_elect(bar(B_Q), C::kQBytes);
+    for (int t = 0; t < 2; ++t)
+      for (int b = 0; b < C::kBoxes; ++b)
+        tma_load_2d_elect(smem_addr(sQ + (t * C::kBoxes + b) * C::kBoxBytes), &tm_q, it.h * DH + b * 64,
+                          it.q_buf_row0 + t * 128, bar(B_Q));
+    KIter ki;
+    make_iter(it, ki);
+    KTile kt;
+    uint32_t c = 0;
+    bool ok = true;
+    while (ok && ki.next(kt)) {
+      for (int w = 0; w < 2 && ok; ++w) {
+        const int slot = c % C::kStages;
+        const uint32_t ph = (c / C::kStages) & 1u;
+        ok = mbar_wait_warp(bar(B_EMPTY + slot), ph ^ 1u, abort_flag, err);
+        if (!ok) break;
+        mbar_arrive_expect_tx_elect(bar(B_FULL + slot), C::kTileBytes);
+        const CUtensorMap* m = w == 0 ? &tm_k : &tm_v;
         for (int b = 0; b < C::kBoxes; ++b)
-          tma_load_2d(smem_addr(sQ + (t * C::kBoxes + b) * C::kBoxBytes), &tm_q, it.h * DH + b * 64,
-                      it.q_buf_row0 + t * 128, bar(B_Q));
-      KIter ki;
-      make_iter(it, ki);
-      KTile kt;
-      uint32_t c = 0;
-      bool ok = true;
-      while (ok && ki.next(kt)) {
-        for (int w = 0; w < 2 && ok; ++w) {
-          const int slot = c % C::kStages;
-          const uint32_t ph = (c / C::kStages) & 1u;
-          ok = mbar_wait(bar(B_EMPTY + slot), ph ^ 1u, abort_flag, err);
-          if (!ok) break;
-          mbar_arrive_expect_tx(bar(B_FULL + slot), C::kTileBytes);
-          const CUtensorMap* m = w == 0 ? &tm_k : &tm_v;
-          for (int b = 0; b < C::kBoxes; ++b)
-            tma_load_2d(smem_addr(sKV + slot * C::kTileBytes + b * C::kBoxBytes), m, it.hk * DH + b * 64,
-                        kt.buf_row, bar(B_FULL + slot));
-          ++c;
-        }
+          tma_load_2d_elect(smem_addr(sKV + slot * C::kTileBytes + b * C::kBoxBytes), m, it.hk * DH + b * 64,
+                            kt.buf_row, bar(B_FULL + slot));
+        ++c;
       }
-      // Drain: make sure every copy this thread issued has landed before the
-      // CTA can exit (only matters after an abort).
-      const uint32_t first = c > (uint32_t)C::kStages ? c - C::kStages : 0u;
-      for (uint32_t i = first; i < c; ++i)
-        mbar_wait(bar(B_FULL + i % C::kStages), (i / C::kStages) & 1u, abort_flag, nullptr, 1000000000ull);
-      mbar_wait(bar(B_Q), 0, abort_flag, nullptr, 1000000000ull);
     }
+    // Drain: make sure every copy issued here has landed before the CTA can
+    // exit (only matters after an abort).
+    const uint32_t first = c > (uint32_t)C::kStages ? c - C::kStages : 0u;
+    for (uint32_t i = first; i < c; ++i)
+      mbar_wait_warp(bar(B_FULL + i % C::kStages), (i / C::kStages) & 1u, abort_flag, nullptr, 1000000000ull);
+    mbar_wait_warp(bar(B_Q), 0, abort_flag, nullptr, 1000000000ull);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, DH, true);
-      const uint32_t sq_base = smem_addr(sQ);
-      const uint32_t skv_base = smem_addr(sKV);
-      auto issue_s = [&](int t, int slot) {
+    // The whole warp runs the loop (operands stay warp-uniform); one elected
+    // lane issues each tcgen05.mma / tcgen05.commit.
+    constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false);
+    constexpr uint32_t idesc_pv = idesc_bf16_f32(128, DH, true);
+    uint32_t pc[2] = {0u, 0u};  // P hand-offs consumed per sub-tile
+    const uint32_t sq_base = smem_addr(sQ);
+    const uint32_t skv_base = smem_addr(sKV);
+    auto issue_s = [&](int t, int slot) {
 #pragma unroll
-        for (int kk = 0; kk < DH / 16; ++kk) {
-          const uint32_t box = kk >> 2, koff = (kk & 3) * 32;
-          const uint64_t a =
-              sdesc_sw128(sq_base + (t * C::kBoxes + box) * C::kBoxBytes + koff, 16, 1024);
-          const uint64_t b = sdesc_sw128(skv_base + slot * C::kTileBytes + box * C::kBoxBytes + koff, 16, 1024);
-          tc_mma_ss(tmem + C::col_s(t), a, b, idesc_qk, kk > 0 ? 1u : 0u);
-        }
-      };
-      auto issue_pv = [&](int t, int slot, bool acc) {
+      for (int kk = 0; kk < DH / 16; ++kk) {
+        const uint32_t box = kk >> 2, koff = (kk & 3) * 32;
+        const uint64_t a = sdesc_sw128(sq_base + (t * C::kBoxes + box) * C::kBoxBytes + koff, 16, 1024);
+        const uint64_t b = sdesc_sw128(skv_base + slot * C::kTileBytes + box * C::kBoxBytes + koff, 16, 1024);
+        tc_mma_ss_elect(tmem + C::col_s(t), a, b, idesc_qk, kk > 0 ? 1u : 0u);
+      }
+    };
+    // O_t += P_t V over the 64 keys of half h of the tile
+    auto issue_pv_half = [&](int t, int slot, int h, bool acc) {
 #pragma unroll
-        for (int kk = 0; kk < CP_KV_TILE / 16; ++kk) {
-          const uint64_t b = sdesc_sw128(skv_base + slot * C::kTileBytes + kk * 2048, C::kBoxBytes, 1024);
-          tc_mma_ts(tmem + C::col_o(t), tmem + C::col_s(t) + kk * 8, b, idesc_pv, (acc || kk > 0) ? 1u : 0u);
-        }
-      };
-      auto kslot = [&](int j) { return (2 * j) % C::kStages; };
-      auto kph = [&](int j) { return (uint32_t)(((2 * j) / C::kStages) & 1); };
-      auto vslot = [&](int j) { return (2 * j + 1) % C::kStages; };
-      auto vph = [&](int j) { return (uint32_t)(((2 * j + 1) / C::kStages) & 1); };
+      for (int k4 = 0; k4 < CP_KV_TILE / 32; ++k4) {
+        const int kk = h * (CP_KV_TILE / 32) + k4;
+        const uint64_t b = sdesc_sw128(skv_base + slot * C::kTileBytes + kk * 2048, C::kBoxBytes, 1024);
+        tc_mma_ts_elect(tmem + C::col_o(t), tmem + C::col_s(t) + kk * 8, b, idesc_pv, (acc || kk > 0) ? 1u : 0u);
+      }
+    };
+    // P_t is released in two halves: the first half's MMAs run while the
+    // softmax computes the second half.
+    auto issue_pv = [&](int t, int slot, bool acc) -> bool {
+      for (int h = 0; h < 2; ++h) {
+        if (!mbar_wait_warp(bar(B_P + 2 * t + h), pc[t] & 1u, abort_flag, err)) return false;
+        tc_fence_after();
+        issue_pv_half(t, slot, h, acc);
+      }
+      ++pc[t];
+      return true;
+    };
+    auto kslot = [&](int j) { return (2 * j) % C::kStages; };
+    auto kph = [&](int j) { return (uint32_t)(((2 * j) / C::kStages) & 1); };
+    auto vslot = [&](int j) { return (2 * j + 1) % C::kStages; };
+    auto vph = [&](int j) { return (uint32_t)(((2 * j + 1) / C::kStages) & 1); };
 
-      bool ok = mbar_wait(bar(B_Q), 0, abort_flag, err);
-      KIter ki;
-      make_iter(it, ki);
-      KTile cur, nxt;
-      bool have = ok && ki.next(cur);
-      uint32_t pc[2] = {0u, 0u};
-      bool acc[2] = {false, false};
-      int j = 0;
-      if (have) {
-        ok = mbar_wait(bar(B_FULL + kslot(0)), kph(0), abort_flag, err);
-        if (ok) {
-          tc_fence_after();
-          if (cur.live0) { issue_s(0, kslot(0)); tc_commit(bar(B_S + 0)); }
-          if (cur.live1) { issue_s(1, kslot(0)); tc_commit(bar(B_S + 1)); }
-          tc_commit(bar(B_EMPTY + kslot(0)));
-        }
-        have = ok;
+    bool ok = mbar_wait_warp(bar(B_Q), 0, abort_flag, err);
+    KIter ki;
+    make_iter(it, ki);
+    KTile cur, nxt;
+    bool have = ok && ki.next(cur);
+    bool acc[2] = {false, false};
+    int j = 0;
+    if (have) {
+      ok = mbar_wait_warp(bar(B_FULL + kslot(0)), kph(0), abort_flag, err);
+      if (ok) {
+        tc_fence_after();
+        if (cur.live0) { issue_s(0, kslot(0)); tc_commit_elect(bar(B_S + 0)); }
+        if (cur.live1) { issue_s(1, kslot(0)); tc_commit_elect(bar(B_S + 1)); }
+        tc_commit_elect(bar(B_EMPTY + kslot(0)));
       }
-      while (have) {
-        const bool hn = ki.next(nxt);
-        if (!(ok = mbar_wait(bar(B_FULL + vslot(j)), vph(j), abort_flag, err))) break;
-        if (cur.live0) {
-          if (!(ok = mbar_wait(bar(B_P + 0), pc[0] & 1u, abort_flag, err))) break;
-          ++pc[0];
-          tc_fence_after();
-          issue_pv(0, vslot(j), acc[0]);
-          acc[0] = true;
-        }
-        if (hn) {
-          if (!(ok = mbar_wait(bar(B_FULL + kslot(j + 1)), kph(j + 1), abort_flag, err))) break;
-          if (nxt.live0) { issue_s(0, kslot(j + 1)); tc_commit(bar(B_S + 0)); }
-        }
-        if (cur.live1) {
-          if (!(ok = mbar_wait(bar(B_P + 1), pc[1] & 1u, abort_flag, err))) break;
-          ++pc[1];
-          tc_fence_after();
-          issue_pv(1, vslot(j), acc[1]);
-          acc[1] = true;
-        }
-        tc_commit(bar(B_EMPTY + vslot(j)));
-        if (hn) {
-          if (nxt.live1) { issue_s(1, kslot(j + 1)); tc_commit(bar(B_S + 1)); }
-          tc_commit(bar(B_EMPTY + kslot(j + 1)));
-        }
-        cur = nxt;
-        have = hn;
-        ++j;
-      }
-      tc_commit(bar(B_O + 0));
-      tc_commit(bar(B_O + 1));
-      // Wait for every MMA issued here before TMEM and shared memory go away.
-      tc_commit(bar(B_DRAIN));
-      mbar_wait(bar(B_DRAIN), 0, abort_flag, nullptr, 1000000000ull);
+      have = ok;
     }
-  } else if (warp >= 4) {
+    while (have) {
+      const bool hn = ki.next(nxt);
+      if (!(ok = mbar_wait_warp(bar(B_FULL + vslot(j)), vph(j), abort_flag, err))) break;
+      if (cur.live0) {
+        if (!(ok = issue_pv(0, vslot(j), acc[0]))) break;
+        acc[0] = true;
+      }
+      if (hn) {
+        if (!(ok = mbar_wait_warp(bar(B_FULL + kslot(j + 1)), kph(j + 1), abort_flag, err))) break;
+        if (nxt.live0) { issue_s(0, kslot(j + 1)); tc_commit_elect(bar(B_S + 0)); }
+      }
+      if (cur.live1) {
+        if (!(ok = issue_pv(1, vslot(j), acc[1]))) break;
+        acc[1] = true;
+      }
+      tc_commit_elect(bar(B_EMPTY + vslot(j)));
+      if (hn) {
+        if (nxt.live1) { issue_s(1, kslot(j + 1)); tc_commit_elect(bar(B_S + 1)); }
+        tc_commit_elect(bar(B_EMPTY + kslot(j + 1)));
+      }
+      cur = nxt;
+      have = hn;
+      ++j;
+    }
+    tc_commit_elect(bar(B_O + 0));
+    tc_commit_elect(bar(B_O + 1));
+    // Wait for every MMA issued here before TMEM and shared memory go away.
+    tc_commit_elect(bar(B_DRAIN));
+    mbar_wait_warp(bar(B_DRAIN), 0, abort_flag, nullptr, 1000000000ull);
+  }
+  } else {
+    regs_inc<216>();
     // ------------------------------------------------------------ softmax
     const int t = (warp - 4) >> 2;
     const int quarter = warp & 3;
@@ -369,13 +392,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int full_lo = t == 0 ? it.full_lo[0] : it.full_lo[1];
     const int full_hi = t == 0 ? it.full_hi[0] : it.full_hi[1];
 
+    // Running state of this row (log2 domain, scores already scaled):
+    //   m_used  reference the accumulated O and l are relative to
+    //   l       sum of 2^(x - m_used) over the keys seen so far
+    //   pend    factor O still has to be multiplied by (lazy rescale)
     float m_used = -CUDART_INF_F;
     float l = 0.f;
+    float pend = 1.f;
     uint32_t n_tiles = 0;
     bool ok = true;
     KIter ki;
     make_iter(it, ki);
     KTile kt;
+    const uint64_t c2 = f2_pack(scale_log2, scale_log2);
+    // O <- O * f for this warp's 32 rows (warp-collective)
+    auto rescale_o = [&](float f) {
+#pragma unroll 1
+      for (int ch = 0; ch < DH / 32; ++ch) {
+        uint32_t o[32];
+        tmem_ld32(tO + ch * 32, o);
+        tc_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+        tmem_st32(tO + ch * 32, o);
+      }
+    };
     while (ki.next(kt)) {
       if (!(t == 0 ? kt.live0 : kt.live1)) continue;
       ok = mbar_wait(bar(B_S + t), n_tiles & 1u, abort_flag, err);
@@ -396,52 +437,96 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < 128; ++c)
           if (c < clo || c > chi) s[c] = __float_as_uint(-CUDART_INF_F);
       }
-      float mx0 = -CUDART_INF_F, mx1 = -CUDART_INF_F, mx2 = -CUDART_INF_F, mx3 = -CUDART_INF_F;
-#pragma unroll
-      for (int c = 0; c < 128; c += 4) {
-        mx0 = fmaxf(mx0, __uint_as_float(s[c + 0]));
-        mx1 = fmaxf(mx1, __uint_as_float(s[c + 1]));
-        mx2 = fmaxf(mx2, __uint_as_float(s[c + 2]));
-        mx3 = fmaxf(mx3, __uint_as_float(s[c + 3]));
+      // S(j) is complete, hence so is PV(j-1): apply a pending rescale of O
+      // before P(j) is released.
+      if (__any_sync(0xffffffffu, pend != 1.f)) {
+        rescale_o(pend);
+        pend = 1.f;
       }
-      const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * scale_log2;
-      const bool need = m_tile > m_used + 8.0f;
-      float alpha = 1.f;
-      if (need) {
-        alpha = ex2_approx(m_used - m_tile);
-        m_used = m_tile;
-        l *= alpha;
-      }
-      const float neg_ref = (m_used == -CUDART_INF_F) ? 0.f : -m_used;
-      float ls0 = 0.f, ls1 = 0.f;
+      // Reference for this tile: the running one.  A row that has seen no
+      // admitted key yet takes the exact maximum of this tile first.
+      float ref = m_used;
+      if (__any_sync(0xffffffffu, ref == -CUDART_INF_F)) {
+        float a = -CUDART_INF_F, b = -CUDART_INF_F;
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pk[32];
+        for (int c = 0; c < 128; c += 4) {
+          a = max3f(a, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+          b = max3f(b, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
+        }
+        if (ref == -CUDART_INF_F) ref = fmaxf(a, b) * scale_log2;
+      }
+      uint32_t pk[32];
+      uint64_t lsum = f2_pack(0.f, 0.f);
+      // P = 2^(x - ref) for columns [64h, 64h + 64), packed to bf16 pairs.
+      // On tiles without masked entries every kPolyEvery-th column pair uses
+      // the FMA-pipe exp2 so that the MUFU unit is not the bottleneck.
+      auto exp_half = [&](int h) {
+        const float nr = ref == -CUDART_INF_F ? 0.f : -ref;
+        const uint64_t nr2 = f2_pack(nr, nr);
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(s[half * 64 + 2 * c]), scale_log2, neg_ref));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(s[half * 64 + 2 * c + 1]), scale_log2, neg_ref));
-          ls0 += p0;
-          ls1 += p1;
+          const uint64_t x = f2_fma(f2_pack(__uint_as_float(s[h * 64 + 2 * c]), __uint_as_float(s[h * 64 + 2 * c + 1])),
+                                    c2, nr2);
+          float p0, p1;
+          if (kPolyEvery > 0 && (c % kPolyEvery) == kPolyEvery - 1 && full) {
+            f2_unpack(exp2_poly_x2(x), p0, p1);
+          } else {
+            float x0, x1;
+            f2_unpack(x, x0, x1);
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
+          }
+          lsum = f2_add(lsum, f2_pack(p0, p1));
           pk[c] = pack_bf16x2(p0, p1);
         }
-        tmem_st32(tS + half * 32, pk);
-      }
-      l += ls0 + ls1;
-      if (n_tiles > 0 && __any_sync(0xffffffffu, need)) {
-#pragma unroll 1
-        for (int ch = 0; ch < DH / 32; ++ch) {
-          uint32_t o[32];
-          tmem_ld32(tO + ch * 32, o);
-          tc_wait_ld();
+      };
+      exp_half(0);
+      // Tile maximum, checked before the first half of P is released.
+      float ma = -CUDART_INF_F, mb = -CUDART_INF_F;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(tO + ch * 32, o);
-        }
+      for (int c = 0; c < 128; c += 4) {
+        ma = max3f(ma, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+        mb = max3f(mb, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
       }
+      const float mt = fmaxf(ma, mb) * scale_log2;
+      // Guard: P must stay far from the bf16 / fp32 range limits.  A row whose
+      // tile maximum exceeds the reference by more than 2^64 re-bases now
+      // (rescaling what O and l hold) and recomputes its P.
+      const bool over = mt > ref + 64.f;
+      if (__any_sync(0xffffffffu, over)) {
+        float f = 1.f;
+        if (over) {
+          f = ex2_approx(ref - mt);
+          ref = mt;
+          l *= f;
+        }
+        if (n_tiles > 0) rescale_o(f);
+        lsum = f2_pack(0.f, 0.f);
+        exp_half(0);
+      }
+      tmem_st32(tS + 0, pk);
       tc_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(B_P + t));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_P + 2 * t + 0));
+      exp_half(1);
+      tmem_st32(tS + 32, pk);
+      tc_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_P + 2 * t + 1));
+      float l0, l1;
+      f2_unpack(lsum, l0, l1);
+      l += l0 + l1;
+      m_used = ref;
+      // Lazy re-basing: move the reference only when the tile maximum is
+      // more than 2^8 above it; O follows at the start of the next tile.
+      if (mt > m_used + 8.f) {
+        const float f = ex2_approx(m_used - mt);
+        pend = f;
+        l *= f;
+        m_used = mt;
+      }
       ++n_tiles;
     }
     if (ok) {
@@ -453,7 +538,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const cp_pair_desc* pd = it.pd;
       const int orow = it.out_row0 + grow;
       float* op = pd->o + ((size_t)orow * plan.hq + it.h) * DH;
-      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      const float inv_l = l > 0.f ? pend / l : 0.f;
       if (n_tiles > 0) {
 #pragma unroll 1
         for (int ch = 0; ch < DH / 32; ++ch) {

@@ -19,7 +19,7 @@
 #include <cstdio>
 #include <mutex>
 
-#include "../../include/cp_attn.h"
+#include "cp_attn.h"
 
 namespace cp {
 void set_error_message(const char* msg);

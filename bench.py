@@ -43,7 +43,11 @@ METRIC = "ring-attn fwd TFLOP/s & % BF16 tensor peak; a2a-permute GB/s % HBM"
 # DRAM traffic per launch of the block-attention kernel from an ncu capture,
 # keyed by the hash of the kernel source it was taken on (null once the
 # kernel changes).  Filled from profiles/ summaries.
-ATTN_TRAFFIC = {}
+ATTN_TRAFFIC = {
+    # profiles/attn_fwd_kernel_ring_contig_32k.md: 2.01 GB read + 1.33 GB written
+    # per launch on the 32K-token contiguous workload (one-pass capture).
+    ("e26710632bba45c5", "ring_contig_32k", 32768): 3.34e9,
+}
 
 
 def src_hash(path):
@@ -388,8 +392,8 @@ def run_ours(args, ws, rank, local):
     value = w["flops"] * ws / (ms_step * 1e-3) / 1e12
     attn_avg = statistics.mean(attn_ms)
     attn_tf = w["flops"] / (attn_avg * 1e-3) / 1e12
-    traffic = ATTN_TRAFFIC.get(src_hash(os.path.join(ROOT, "context_exact_attention_step_b200", "csrc",
-                                                     "attn_fwd.cu")))
+    traffic = ATTN_TRAFFIC.get((src_hash(os.path.join(ROOT, "context_exact_attention_step_b200", "csrc",
+                                                      "attn_fwd.cu")), w["name"], w["S"]))
     e2e_ms, h2d, d2h = time_e2e(w, args.e2e_steps)
     e2e_ms = max_over_ranks(e2e_ms, ws)
     perm = time_permute() if not args.no_permute else None

@@ -24,7 +24,7 @@ EXPORTS = [
     "cp_ring_attn_workspace_size", "cp_ring_attn_fwd", "cp_ulysses_permute", "cp_zigzag_reorder",
     "cp_ulysses_attn_workspace_size", "cp_ulysses_attn_fwd", "cp_ring_schedule", "cp_count_live_pairs",
     "cp_device_error", "cp_kernel_launch_count", "cp_set_profile_events",
-    "cp_ring_attn_fwd_noalloc",
+    "cp_ring_attn_fwd_noalloc", "cp_selftest_wait_timeout",
 ]
 
 
@@ -88,6 +88,8 @@ def lib():
     L.cp_kernel_launch_count.argtypes = [ctypes.POINTER(ctypes.c_uint64)]
     L.cp_set_profile_events.restype = i32
     L.cp_set_profile_events.argtypes = [vp, vp, vp]
+    L.cp_selftest_wait_timeout.restype = i32
+    L.cp_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp]
     L.cp_device_error.restype = i32
     L.cp_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32), i32]
     _lib = L

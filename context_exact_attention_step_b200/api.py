@@ -272,6 +272,11 @@ def set_profile_events(attn_begin=None, attn_end=None, merge_end=None):
     check(lib().cp_set_profile_events(h(attn_begin), h(attn_end), h(merge_end)))
 
 
+def selftest_wait_timeout(timeout_ns=1_000_000, stream=None):
+    """Launch the bounded-wait self-test (see cp_selftest_wait_timeout)."""
+    check(lib().cp_selftest_wait_timeout(int(timeout_ns), _stream(stream)))
+
+
 def device_error(clear=True) -> int:
     bits = ctypes.c_uint32(0)
     check(lib().cp_device_error(ctypes.byref(bits), 1 if clear else 0))

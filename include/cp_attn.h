@@ -219,6 +219,13 @@ cp_status cp_ring_schedule(int S, int P, cp_layout layout, cp_mask mask, const i
  * the causal-effective FLOP count 4 * dh * hq * pairs.  Host only. */
 cp_status cp_count_live_pairs(int S, cp_mask mask, const int32_t* cu_seqlens_host, int n_docs, int64_t* pairs);
 
+/* Self-test of failure detection: launches one CTA that waits on a barrier
+ * nothing ever arrives on.  The bounded wait gives up after timeout_ns
+ * (0 < timeout_ns <= 10 s), sets bit 0 of the device error word (read it with
+ * cp_device_error after synchronising) and returns; the CUDA context stays
+ * usable.  Used by the tests; the pages have no counterpart. */
+cp_status cp_selftest_wait_timeout(uint64_t timeout_ns, void* stream);
+
 /* Reads (and, if clear != 0, resets) the device error word of the current
  * device: 0 = no kernel gave up waiting; bit 0 = a bounded wait timed out.
  * Synchronous. */

@@ -92,14 +92,14 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// bf16 matrix of `rows` rows x `row_elems` elements, 128-row x 64-column
+// bf16 matrix of `rows` rows x `row_elems` elements, box_rows-row x 64-column
 // boxes with 128-byte swizzle (the canonical K-major tcgen05 operand layout).
-cp_status make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t row_elems) {
+cp_status make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t row_elems, uint32_t box_rows) {
   auto fn = encode_fn();
   if (!fn) return fail(CP_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   cuuint64_t dims[2] = {(cuuint64_t)row_elems, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)row_elems * 2};
-  cuuint32_t box[2] = {64, 128};
+  cuuint32_t box[2] = {64, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -140,9 +140,10 @@ cp_status run_pairs(const void* q, const void* k, const void* v, int64_t q_rows,
                     const std::vector<PairIn>& pairs, cudaStream_t st) {
   CUtensorMap tq, tk, tv;
   cp_status s;
-  if ((s = make_map(&tq, q, q_rows, (int64_t)hq * dh)) != CP_OK) return s;
-  if ((s = make_map(&tk, k, k_rows, (int64_t)hkv * dh)) != CP_OK) return s;
-  if ((s = make_map(&tv, v, k_rows, (int64_t)hkv * dh)) != CP_OK) return s;
+  // query boxes: one 128-row MMA tile; key/value boxes: one CP_KV_TILE-row tile
+  if ((s = make_map(&tq, q, q_rows, (int64_t)hq * dh, 128)) != CP_OK) return s;
+  if ((s = make_map(&tk, k, k_rows, (int64_t)hkv * dh, CP_KV_TILE)) != CP_OK) return s;
+  if ((s = make_map(&tv, v, k_rows, (int64_t)hkv * dh, CP_KV_TILE)) != CP_OK) return s;
   uint32_t* err = nullptr;
   if ((s = err_word(&err)) != CP_OK) return s;
 

@@ -7,11 +7,11 @@
 #include <stdint.h>
 
 #define CP_MAX_SEGS 4        // row segments per side of one block pair
-#define CP_MAX_PAIRS 48      // block pairs per attention launch
+#define CP_MAX_PAIRS 64      // block pairs per attention launch
 #define CP_MAX_TASKS 32      // merge tasks per merge launch
 #define CP_MAX_INPUTS 192    // merge inputs per merge launch
 #define CP_Q_TILE 256        // query rows per CTA (two 128-row MMA tiles)
-#define CP_KV_TILE 128       // key/value rows per pipeline stage
+#define CP_KV_TILE 128       // key/value rows per pipeline stage (and per S tile)
 
 // A run of consecutive buffer rows whose global token positions are also
 // consecutive.  buf_row: first row in the Q/K/V buffer; pos: global position

@@ -7,7 +7,7 @@
 // each partial carries its own max and denominator folded into LSE_i, and the
 // fold rescales each partial's normalised O by its share of the total
 // denominator.  Partials whose LSE_i is -inf hold no admitted key for that row;
-// they get weight 0 and their O is never read.  All arithmetic is fp32.
+// they get weight 0 and their O is never combined.  All arithmetic is fp32.
 //
 // One group of dh/4 threads handles one (row, head): every thread owns four
 // consecutive columns and moves them with 16-byte loads and stores, so a warp
@@ -28,6 +28,7 @@ template <int DH>
 __global__ void __launch_bounds__(256) lse_merge_kernel(const __grid_constant__ cp_merge_plan plan) {
   constexpr int TPI = DH / 4;        // threads per (row, head)
   constexpr int IPB = 256 / TPI;     // (row, head) items per block
+  constexpr int U = 4;               // partials whose loads are in flight together
   const cp_merge_task& task = plan.tasks[blockIdx.y];
   const int item = blockIdx.x * IPB + threadIdx.x / TPI;
   const int sub = threadIdx.x % TPI;
@@ -38,48 +39,49 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(const __grid_constant__ 
 
   const cp_merge_input* in = plan.inputs + task.in_begin;
   const int n = task.n_in;
-  float m = -CUDART_INF_F;
-  for (int i = 0; i < n; ++i) {
-    const float li = __ldg(in[i].lse + (size_t)head * in[i].lse_ld + in[i].row0 + row);
-    m = fmaxf(m, li);
-  }
+  // Single pass with a running maximum: the LSE and O loads of U partials
+  // are issued together (no load waits on another), then folded.
+  float m = -CUDART_INF_F, tot = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  float tot = 0.f;
-  if (m != -CUDART_INF_F) {
-    int i = 0;
-    // four partials per round keeps four 16-byte loads in flight per thread
-    for (; i + 4 <= n; i += 4) {
-      float w[4];
-      float4 o[4];
+  for (int i0 = 0; i0 < n; i0 += U) {
+    float li[U];
+    float4 o[U];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const cp_merge_input& x = in[i + u];
-        const float li = __ldg(x.lse + (size_t)head * x.lse_ld + x.row0 + row);
-        w[u] = li == -CUDART_INF_F ? 0.f : expf(li - m);
-        o[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (w[u] > 0.f)
-          o[u] = __ldcs(reinterpret_cast<const float4*>(x.o + ((size_t)(x.row0 + row) * h + head) * DH) + sub);
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        tot += w[u];
-        acc.x = fmaf(w[u], o[u].x, acc.x);
-        acc.y = fmaf(w[u], o[u].y, acc.y);
-        acc.z = fmaf(w[u], o[u].z, acc.z);
-        acc.w = fmaf(w[u], o[u].w, acc.w);
+    for (int u = 0; u < U; ++u) {
+      li[u] = -CUDART_INF_F;
+      o[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (i0 + u < n) {
+        const cp_merge_input& x = in[i0 + u];
+        li[u] = __ldg(x.lse + (size_t)head * x.lse_ld + x.row0 + row);
+        o[u] = __ldcs(reinterpret_cast<const float4*>(x.o + ((size_t)(x.row0 + row) * h + head) * DH) + sub);
       }
     }
-    for (; i < n; ++i) {
-      const cp_merge_input& x = in[i];
-      const float li = __ldg(x.lse + (size_t)head * x.lse_ld + x.row0 + row);
-      if (li == -CUDART_INF_F) continue;
-      const float w = expf(li - m);
-      const float4 o = __ldcs(reinterpret_cast<const float4*>(x.o + ((size_t)(x.row0 + row) * h + head) * DH) + sub);
-      tot += w;
-      acc.x = fmaf(w, o.x, acc.x);
-      acc.y = fmaf(w, o.y, acc.y);
-      acc.z = fmaf(w, o.z, acc.z);
-      acc.w = fmaf(w, o.w, acc.w);
+    float mr = m;
+#pragma unroll
+    for (int u = 0; u < U; ++u) mr = fmaxf(mr, li[u]);
+    if (mr != -CUDART_INF_F) {
+      if (mr > m) {
+        const float f = m == -CUDART_INF_F ? 0.f : expf(m - mr);
+        tot *= f;
+        acc.x *= f;
+        acc.y *= f;
+        acc.z *= f;
+        acc.w *= f;
+        m = mr;
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        // a partial with LSE = -inf has no admitted key: weight 0, and its O
+        // (possibly not a number) is never combined
+        if (li[u] != -CUDART_INF_F) {
+          const float w = expf(li[u] - m);
+          tot += w;
+          acc.x = fmaf(w, o[u].x, acc.x);
+          acc.y = fmaf(w, o[u].y, acc.y);
+          acc.z = fmaf(w, o[u].z, acc.z);
+          acc.w = fmaf(w, o[u].w, acc.w);
+        }
+      }
     }
   }
   const float inv = tot > 0.f ? 1.f / tot : 0.f;

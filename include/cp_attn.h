@@ -107,7 +107,8 @@ cp_status cp_block_attn_fwd(const void* q, const void* k, const void* v, cp_dtyp
  * cp_lse_merge -- fold n_parts partial results over the same rows:
  *   LSE = ln sum_i exp(LSE_i),  O = sum_i exp(LSE_i - LSE) * O_i,
  * in fp32; partials with LSE_i = -inf for a row contribute nothing there (their
- * O is not read); rows where every LSE_i is -inf get O = 0, LSE = -inf.  The
+ * O is never combined, so it may hold anything, NaN included); rows where every
+ * LSE_i is -inf get O = 0, LSE = -inf.  The
  * block-granular form of the online-softmax recurrence ("序列並行" concept page
  * (compassingai), 技術原理 §二).
  *

@@ -95,3 +95,11 @@ def test_documents_noncausal():
 def test_long_pair_many_tiles():
     err_o, err_l = run_case([(0, 2048)], [(0, 2048)], hq=2, hkv=1)
     assert err_o < 5e-3 and err_l < 1e-4
+
+
+def test_four_chunks_per_side():
+    # up to CP_MAX_CHUNKS segments on each side, out of position order
+    qc = [(900, 100), (0, 50), (300, 130), (2000, 40)]
+    kc = [(0, 200), (250, 300), (880, 77), (1990, 60)]
+    run_case(qc, kc, hq=2, hkv=1)
+    run_case(qc, kc, hq=2, hkv=1, causal=False)

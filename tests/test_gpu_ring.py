@@ -139,3 +139,30 @@ def test_full_size_ulysses_gqa_128k():
     want_o, want_l = ref.attention(f64(q[torch.from_numpy(rows)]), f64(k), f64(v), causal=True, qpos=rows)
     idx = torch.from_numpy(rows).cuda()
     compare(o[idx], lse[:, idx], want_o, want_l, what="full ulysses")
+
+
+# ----------------------------------------------------------- more shapes
+@pytest.mark.parametrize("layout", ["contiguous", "zigzag"])
+def test_sixteen_ranks_split_launches(layout):
+    # P = 16: up to 256 block pairs, more than one attention launch
+    ring_case(4096, 2, 2, 64, 16, layout)
+
+
+def test_gqa_inside_the_ring():
+    ring_case(2048, 8, 2, 128, 4, "zigzag")
+
+
+def test_varlen_gqa_contiguous():
+    S = 3072
+    lens = synth.doc_lengths(S, 100, 900, seed=9)
+    ring_case(S, 4, 2, 64, 4, "contiguous", cu=synth.cu_seqlens_from_lengths(lens).tolist())
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_ulysses_dh64(causal):
+    S, hq, hkv, dh, P = 1024, 8, 8, 64, 4
+    q, k, v = synth.qkv(S, hq, hkv, dh)
+    o, lse = api.ulysses_attn_fwd(q.cuda(), k.cuda(), v.cuda(), P, causal=causal)
+    torch.cuda.synchronize()
+    want_o, want_l = ref.attention(f64(q), f64(k), f64(v), causal=causal)
+    compare(o, lse, want_o, want_l, what=f"ulysses dh64 causal={causal}")

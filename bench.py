@@ -181,18 +181,19 @@ def make_workload(name, seq_len=None):
         cu_dev = torch.tensor(cu, dtype=torch.int32, device=dev) if cu is not None else None
         ws = torch.empty(max(256, api.ring_attn_workspace_size(S, hq, hkv, dh, P, layout, True, dtype, cu)),
                          device=dev, dtype=torch.uint8)
-        if layout == "zigzag":
+        if layout in ("zigzag", "striped"):
             qz, kz, vz = (torch.empty_like(t) for t in (qd, kd, vd))
             oz = torch.empty_like(o)
             lz = torch.empty_like(lse)
+            reorder = api.zigzag_reorder if layout == "zigzag" else api.striped_reorder
 
             def step():
-                api.zigzag_reorder(qd, P, out=qz)
-                api.zigzag_reorder(kd, P, out=kz)
-                api.zigzag_reorder(vd, P, out=vz)
+                reorder(qd, P, out=qz)
+                reorder(kd, P, out=kz)
+                reorder(vd, P, out=vz)
                 api.ring_attn_fwd(qz, kz, vz, P, layout, True, cu, cu_dev, o=oz, lse=lz, workspace=ws)
-                api.zigzag_reorder(oz, P, inverse=True, out=o)
-                api.zigzag_reorder(lz, P, inverse=True, seq_dim=1, out=lse)
+                reorder(oz, P, inverse=True, out=o)
+                reorder(lz, P, inverse=True, seq_dim=1, out=lse)
         else:
             def step():
                 api.ring_attn_fwd(qd, kd, vd, P, layout, True, cu, cu_dev, o=o, lse=lse, workspace=ws)

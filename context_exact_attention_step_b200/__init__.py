@@ -11,6 +11,7 @@ from .api import (  # noqa: F401
     device_error,
     kernel_launch_count,
     set_profile_events,
+    striped_reorder,
     lse_merge,
     ring_attn_fwd,
     ring_attn_workspace_size,

@@ -12,7 +12,7 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libcp_attn
 CP_OK, CP_ERR_INVALID_ARG, CP_ERR_UNSUPPORTED, CP_ERR_ALIGNMENT, CP_ERR_WORKSPACE, CP_ERR_CUDA = range(6)
 CP_BF16, CP_FP32 = 0, 1
 CP_MASK_NONE, CP_MASK_CAUSAL = 0, 1
-CP_LAYOUT_CONTIGUOUS, CP_LAYOUT_ZIGZAG = 0, 1
+CP_LAYOUT_CONTIGUOUS, CP_LAYOUT_ZIGZAG, CP_LAYOUT_STRIPED = 0, 1, 2
 CP_SEQ_TO_HEAD, CP_HEAD_TO_SEQ = 0, 1
 CP_MAX_CHUNKS = 4
 
@@ -24,7 +24,7 @@ EXPORTS = [
     "cp_ring_attn_workspace_size", "cp_ring_attn_fwd", "cp_ulysses_permute", "cp_zigzag_reorder",
     "cp_ulysses_attn_workspace_size", "cp_ulysses_attn_fwd", "cp_ring_schedule", "cp_count_live_pairs",
     "cp_device_error", "cp_kernel_launch_count", "cp_set_profile_events",
-    "cp_ring_attn_fwd_noalloc", "cp_selftest_wait_timeout",
+    "cp_ring_attn_fwd_noalloc", "cp_selftest_wait_timeout", "cp_striped_reorder",
 ]
 
 
@@ -73,6 +73,8 @@ def lib():
                                            vp, vp, vp]
     L.cp_ulysses_permute.restype = i32
     L.cp_ulysses_permute.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, vp]
+    L.cp_striped_reorder.restype = i32
+    L.cp_striped_reorder.argtypes = [vp, vp, i32, i32, i32, i32, i32, vp]
     L.cp_zigzag_reorder.restype = i32
     L.cp_zigzag_reorder.argtypes = [vp, vp, i32, i32, i32, i32, i32, vp]
     L.cp_ulysses_attn_workspace_size.restype = i32

@@ -16,7 +16,8 @@ import torch
 from . import _lib
 from ._lib import check, cp_chunk, lib
 
-_LAYOUTS = {"contiguous": _lib.CP_LAYOUT_CONTIGUOUS, "zigzag": _lib.CP_LAYOUT_ZIGZAG}
+_LAYOUTS = {"contiguous": _lib.CP_LAYOUT_CONTIGUOUS, "zigzag": _lib.CP_LAYOUT_ZIGZAG,
+            "striped": _lib.CP_LAYOUT_STRIPED}
 
 
 def _vp(t: Optional[torch.Tensor]):
@@ -206,6 +207,24 @@ def zigzag_reorder(x, P, inverse=False, seq_dim=0, out=None, stream=None):
     if out is None:
         out = torch.empty_like(x)
     check(lib().cp_zigzag_reorder(_vp(x), _vp(out), P, S, batch, row_bytes, 1 if inverse else 0, _stream(stream)))
+    return out
+
+
+def striped_reorder(x, P, inverse=False, seq_dim=0, out=None, stream=None):
+    """Natural <-> rank-major striped order (token t on rank t mod P) along
+    ``seq_dim`` (0 for [S, ...] tensors, 1 for [h, S] LSE tensors)."""
+    _need_cuda("x", x)
+    if seq_dim == 0:
+        batch, S = 1, x.shape[0]
+        row_bytes = x[0].numel() * x.element_size() if x.dim() > 1 else x.element_size()
+    elif seq_dim == 1 and x.dim() == 2:
+        batch, S = x.shape
+        row_bytes = x.element_size()
+    else:
+        raise ValueError("seq_dim must be 0, or 1 for a 2-D tensor")
+    if out is None:
+        out = torch.empty_like(x)
+    check(lib().cp_striped_reorder(_vp(x), _vp(out), P, S, batch, row_bytes, 1 if inverse else 0, _stream(stream)))
     return out
 
 

@@ -29,6 +29,8 @@ cudaError_t launch_ulysses(const void* in, void* out, int P, int n, size_t chunk
 cudaError_t launch_zigzag(const void* in, void* out, int P, int batch, size_t chunk_bytes, int inverse,
                           cudaStream_t st);
 cudaError_t launch_f32_to_bf16(const float* in, void* out, size_t n, cudaStream_t st);
+cudaError_t launch_striped(const void* in, void* out, int P, int S, int batch, size_t row_bytes, int inverse,
+                           cudaStream_t st);
 std::atomic<uint64_t>& launch_counter();
 }  // namespace cp
 
@@ -341,8 +343,10 @@ static cp_status ring_check(int S, int hq, int hkv, int dh, int P, cp_layout lay
   if ((s = check_common(hq, hkv, dh)) != CP_OK) return s;
   if (P < 1 || P > 16) return fail(CP_ERR_UNSUPPORTED, "P = %d (supported 1..16)", P);
   if (S <= 0 || S >= (1 << 30)) return fail(CP_ERR_INVALID_ARG, "S = %d", S);
-  if (layout != CP_LAYOUT_CONTIGUOUS && layout != CP_LAYOUT_ZIGZAG)
+  if (layout != CP_LAYOUT_CONTIGUOUS && layout != CP_LAYOUT_ZIGZAG && layout != CP_LAYOUT_STRIPED)
     return fail(CP_ERR_INVALID_ARG, "unknown layout %d", (int)layout);
+  if (layout == CP_LAYOUT_STRIPED && n_docs > 0)
+    return fail(CP_ERR_UNSUPPORTED, "the striped layout does not take a document mask");
   if (mask != CP_MASK_NONE && mask != CP_MASK_CAUSAL) return fail(CP_ERR_INVALID_ARG, "unknown mask %d", (int)mask);
   if (dtype != CP_BF16 && dtype != CP_FP32) return fail(CP_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
   const int div = layout == CP_LAYOUT_ZIGZAG ? 2 * P : P;
@@ -357,8 +361,10 @@ static RingPlan make_ring_plan(int S, int hq, int dh, int P, cp_layout layout, c
     docs.cu = cu_host;
     docs.n = n_docs;
   }
-  return build_ring_plan(S, P, layout == CP_LAYOUT_ZIGZAG ? Layout::Zigzag : Layout::Contiguous,
-                         mask == CP_MASK_CAUSAL, docs, hq, dh);
+  const Layout lay = layout == CP_LAYOUT_ZIGZAG ? Layout::Zigzag
+                     : layout == CP_LAYOUT_STRIPED ? Layout::Striped
+                                                   : Layout::Contiguous;
+  return build_ring_plan(S, P, lay, mask == CP_MASK_CAUSAL, docs, hq, dh);
 }
 
 cp_status cp_ring_attn_workspace_size(int S, int hq, int hkv, int dh, int P, cp_layout layout, cp_mask mask,
@@ -480,6 +486,20 @@ cp_status cp_zigzag_reorder(const void* in, void* out, int P, int S, int batch, 
   const size_t chunk = (size_t)(S / (2 * P)) * row_bytes;
   cudaError_t e = launch_zigzag(in, out, P, batch, chunk, inverse ? 1 : 0, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "zigzag reorder launch");
+  return ok();
+}
+
+cp_status cp_striped_reorder(const void* in, void* out, int P, int S, int batch, int row_bytes, int inverse,
+                             void* stream) {
+  if (!in || !out) return fail(CP_ERR_INVALID_ARG, "in/out is NULL");
+  if (P < 1 || S <= 0 || batch <= 0 || row_bytes <= 0) return fail(CP_ERR_INVALID_ARG, "sizes must be positive");
+  if (S % P != 0) return fail(CP_ERR_INVALID_ARG, "S = %d is not a multiple of P = %d", S, P);
+  const size_t bytes = (size_t)batch * S * row_bytes;
+  const uint8_t *a = static_cast<const uint8_t*>(in), *b = static_cast<const uint8_t*>(out);
+  if (a < b + bytes && b < a + bytes) return fail(CP_ERR_INVALID_ARG, "in and out overlap");
+  cudaError_t e = launch_striped(in, out, P, S, batch, (size_t)row_bytes, inverse ? 1 : 0,
+                                 static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "striped reorder launch");
   return ok();
 }
 

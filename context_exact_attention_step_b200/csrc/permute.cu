@@ -8,6 +8,8 @@
 //  * Zigzag reorder: rank-major layout in which rank i holds chunks i and
 //    2P-1-i of the 2P equal chunks ("长上下文序列并行训练深度解析" (mooersco),
 //    timeline: Striped / zigzag load-balancing reorder), and its inverse.
+//  * Striped reorder: token t on rank t mod P (same timeline, Striped
+//    Attention), and its inverse.
 //  * fp32 -> bf16 round-to-nearest-even conversion of input tensors.
 //
 // Both layout changes move whole runs of >= 256 contiguous bytes (one head
@@ -97,6 +99,30 @@ __global__ void __launch_bounds__(256) zigzag_kernel(const U* __restrict__ in, U
       const size_t u = u0 + i * stride;
       if (u < chunk_units) st_stream(out + dst_base + u, v[i]);
     }
+  }
+}
+
+// Striped layout: rank r holds positions r, r + P, ...; rank-major row
+// r * n + a holds natural row a * P + r (n = S / P).  One CTA row-loop per
+// batch entry; every row is copied with `upr` units.
+template <typename U>
+__global__ void __launch_bounds__(256) striped_kernel(const U* __restrict__ in, U* __restrict__ out, int P, int n,
+                                                      uint32_t upr, int inverse) {
+  const size_t S = (size_t)P * n;
+  const size_t base = (size_t)blockIdx.y * S * upr;
+  const uint32_t total = (uint32_t)(S * upr);
+  for (uint32_t u = blockIdx.x * blockDim.x + threadIdx.x; u < total; u += gridDim.x * blockDim.x) {
+    const uint32_t orow = u / upr;
+    const uint32_t c = u - orow * upr;
+    uint32_t irow;
+    if (!inverse) {  // out row r*n + a <- natural row a*P + r
+      const uint32_t r = orow / n, a = orow - r * n;
+      irow = a * P + r;
+    } else {         // out row a*P + r <- rank-major row r*n + a
+      const uint32_t a = orow / P, r = orow - a * P;
+      irow = r * n + a;
+    }
+    st_stream(out + base + (size_t)orow * upr + c, ld_stream(in + base + (size_t)irow * upr + c));
   }
 }
 
@@ -192,6 +218,32 @@ cudaError_t launch_zigzag(const void* in, void* out, int P, int batch, size_t ch
     case 4: return zigzag_t<uint32_t>(in, out, P, batch, chunk_bytes, inverse, st);
     case 2: return zigzag_t<uint16_t>(in, out, P, batch, chunk_bytes, inverse, st);
     default: return zigzag_t<uint8_t>(in, out, P, batch, chunk_bytes, inverse, st);
+  }
+}
+
+template <typename U>
+static cudaError_t striped_t(const void* in, void* out, int P, int n, int batch, size_t row_bytes, int inverse,
+                            cudaStream_t st) {
+  const uint32_t upr = (uint32_t)(row_bytes / sizeof(U));
+  const size_t total = (size_t)P * n * upr;
+  size_t gx = (total + 255) / 256;
+  const size_t wave = (size_t)num_sms() * 8;
+  if (gx > wave) gx = wave;
+  dim3 grid((unsigned)gx, (unsigned)batch);
+  striped_kernel<U><<<grid, 256, 0, st>>>(static_cast<const U*>(in), static_cast<U*>(out), P, n, upr, inverse);
+  launch_counter()++;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_striped(const void* in, void* out, int P, int S, int batch, size_t row_bytes, int inverse,
+                           cudaStream_t st) {
+  const int n = S / P;
+  switch (unit_bytes(row_bytes, in, out)) {
+    case 16: return striped_t<uint4>(in, out, P, n, batch, row_bytes, inverse, st);
+    case 8: return striped_t<uint2>(in, out, P, n, batch, row_bytes, inverse, st);
+    case 4: return striped_t<uint32_t>(in, out, P, n, batch, row_bytes, inverse, st);
+    case 2: return striped_t<uint16_t>(in, out, P, n, batch, row_bytes, inverse, st);
+    default: return striped_t<uint8_t>(in, out, P, n, batch, row_bytes, inverse, st);
   }
 }
 

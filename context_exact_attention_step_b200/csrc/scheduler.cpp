@@ -41,6 +41,9 @@ std::vector<Seg> shard_segments(int S, int P, Layout layout, int r) {
   if (layout == Layout::Contiguous) {
     const int n = S / P;
     s.push_back({r * n, r * n, n, 0});
+  } else if (layout == Layout::Striped) {
+    const int n = S / P;
+    s.push_back({r * n, 0, n, 0});
   } else {
     const int c = S / (2 * P);
     const int base = r * 2 * c;
@@ -134,6 +137,12 @@ RingPlan build_ring_plan(int S, int P, Layout layout, bool causal, const Docs& d
       pp.t = t;
       pp.j = j;
       pp.k = shard_segments(S, P, layout, j);
+      if (layout == Layout::Striped && j > r) {
+        // Striped: rank r holds positions r + P*a, shard j positions j + P*b.
+        // k <= q  <=>  b <= a for j <= r and b <= a - 1 for j > r, i.e. a
+        // local causal mask whose key positions are shifted by one for j > r.
+        pp.k[0].pos = 1;
+      }
       int out_row = 0;
       for (const Seg& qs : qsegs) {
         int lo = INT_MAX, hi = INT_MIN;

@@ -10,7 +10,7 @@
 
 namespace cp {
 
-enum class Layout { Contiguous = 0, Zigzag = 1 };
+enum class Layout { Contiguous = 0, Zigzag = 1, Striped = 2 };
 
 // Document table on the host (prefix sums; n docs, n + 1 entries), or none.
 struct Docs {
@@ -55,7 +55,9 @@ struct RingPlan {
   std::vector<int64_t> live_all;      // per (r, t)
 };
 
-// Segments of rank r's shard, buf_row absolute (rank-major storage).
+// Segments of rank r's shard, buf_row absolute (rank-major storage).  For the
+// striped layout the positions are per-pair virtual positions (see
+// build_ring_plan), and this returns the shard's rows at position 0.
 std::vector<Seg> shard_segments(int S, int P, Layout layout, int r);
 
 // Admitted (q, k) pairs between position ranges [qa, qa+ql) and [ka, ka+kl).

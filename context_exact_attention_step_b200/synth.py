@@ -66,6 +66,8 @@ CONFIGS = {
                             causal=True, varlen=False, std=0.5, dtype="bf16"),
     "ring_zigzag_64k": dict(S=65536, hq=32, hkv=32, dh=128, P=8, layout="zigzag",
                             causal=True, varlen=False, std=0.5, dtype="bf16"),
+    "ring_striped_64k": dict(S=65536, hq=32, hkv=32, dh=128, P=8, layout="striped",
+                             causal=True, varlen=False, std=0.5, dtype="bf16"),
     "ulysses_gqa_128k": dict(S=131072, hq=32, hkv=8, dh=128, P=8, layout="ulysses",
                              causal=True, varlen=False, std=0.5, dtype="bf16"),
     "varlen_zigzag_128k": dict(S=131072, hq=32, hkv=32, dh=128, P=8, layout="zigzag",

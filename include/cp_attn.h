@@ -47,7 +47,7 @@ typedef enum {
 
 typedef enum { CP_BF16 = 0, CP_FP32 = 1 } cp_dtype;
 typedef enum { CP_MASK_NONE = 0, CP_MASK_CAUSAL = 1 } cp_mask;
-typedef enum { CP_LAYOUT_CONTIGUOUS = 0, CP_LAYOUT_ZIGZAG = 1 } cp_layout;
+typedef enum { CP_LAYOUT_CONTIGUOUS = 0, CP_LAYOUT_ZIGZAG = 1, CP_LAYOUT_STRIPED = 2 } cp_layout;
 typedef enum { CP_SEQ_TO_HEAD = 0, CP_HEAD_TO_SEQ = 1 } cp_dir;
 
 /* A run of consecutive rows of a Q or K/V buffer whose global token
@@ -148,7 +148,10 @@ cp_status cp_ring_attn_workspace_size(int S, int hq, int hkv, int dh, int P, cp_
  *                [r*S/P, (r+1)*S/P).  CP_LAYOUT_CONTIGUOUS: rank r holds
  *                positions [r*S/P, (r+1)*S/P).  CP_LAYOUT_ZIGZAG: rank r holds
  *                chunk r then chunk 2P-1-r of the 2P chunks of S/(2P) tokens
- *                (cp_zigzag_reorder produces this order).
+ *                (cp_zigzag_reorder produces this order).  CP_LAYOUT_STRIPED:
+ *                rank r holds positions r, r+P, r+2P, ... (Striped Attention,
+ *                same timeline; cp_striped_reorder produces this order); not
+ *                combinable with documents (CP_ERR_UNSUPPORTED).
  *   cu_seqlens_host, cu_seqlens_dev  the same document table on host and device
  *                (n_docs + 1 entries; both NULL and n_docs = 0 for none); the
  *                host copy lets the scheduler skip pairs across documents
@@ -188,6 +191,16 @@ cp_status cp_ulysses_permute(const void* in, void* out, int P, int S, int h, int
  */
 cp_status cp_zigzag_reorder(const void* in, void* out, int P, int S, int batch, int row_bytes, int inverse,
                             void* stream);
+
+/*
+ * cp_striped_reorder -- natural token order <-> rank-major striped order
+ * (token t on rank t mod P, rank r's rows in position order: row r*S/P + a
+ * holds position a*P + r).  in/out are [batch][S][row_bytes] byte arrays as
+ * for cp_zigzag_reorder.  inverse = 0: natural -> striped; 1: back.  Bit-exact.
+ * Supported: S % P == 0; in and out must not overlap.
+ */
+cp_status cp_striped_reorder(const void* in, void* out, int P, int S, int batch, int row_bytes, int inverse,
+                             void* stream);
 
 /*
  * cp_ulysses_attn_workspace_size / cp_ulysses_attn_fwd -- the Ulysses path:

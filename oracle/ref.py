@@ -24,7 +24,8 @@ definition itself:
 * ``zigzag_order`` / ``zigzag_reorder`` / ``zigzag_restore`` -- shard i holds
   chunks i and 2P-1-i of the 2P equal chunks ("长上下文序列并行训练深度解析"
   (mooersco) timeline: Striped / zigzag load-balancing reorder; the exact chunk
-  pairing is the plainest balanced reading and is recorded in the design doc).
+  pairing is the plainest balanced reading).  ``striped_order``: token t on
+  rank t mod P (same timeline, Striped Attention).
 * ``ulysses_seq_to_head`` / ``ulysses_head_to_seq`` -- the all-to-all
   transpose [S/P, H, d_h] -> [S, H/P, d_h] (compassingai §三 "Ulysses 的
   AllToAll 轉置"; pwwt.cn §2.3), device i taking head block i.
@@ -116,7 +117,10 @@ def attention(q, k, v, causal=True, cu_seqlens=None, scale=None, qpos=None,
 def shard_positions(S, P, layout, r):
     """Global positions held by virtual rank r, in the order the rank stores
     them.  contiguous: [r*S/P, (r+1)*S/P).  zigzag: chunk r then chunk 2P-1-r
-    of the 2P chunks of S/(2P) tokens."""
+    of the 2P chunks of S/(2P) tokens.  striped: r, r+P, r+2P, ... (token t
+    on rank t mod P)."""
+    if layout == "striped":
+        return np.arange(r, S, P)
     if layout == "contiguous":
         n = S // P
         return np.arange(r * n, (r + 1) * n)
@@ -137,6 +141,12 @@ def zigzag_reorder(x, P, axis=0):
     """Natural order -> rank-major zigzag order (gather along ``axis``)."""
     x = np.asarray(x)
     return np.take(x, zigzag_order(x.shape[axis], P), axis=axis)
+
+
+def striped_order(S, P):
+    """order[i] = natural position of the token stored at row i of the
+    rank-major striped layout."""
+    return np.concatenate([shard_positions(S, P, "striped", r) for r in range(P)])
 
 
 def zigzag_restore(y, P, axis=0):

@@ -87,6 +87,11 @@ def test_ring_rejects_bad_arguments():
     assert _ring(cu=short, n_docs=2) == _lib.CP_ERR_INVALID_ARG     # does not end at S
 
 
+def test_striped_rejects_documents():
+    cu = (ctypes.c_int32 * 3)(0, 600, 1024)
+    assert _ring(layout=_lib.CP_LAYOUT_STRIPED, cu=cu, n_docs=2) == _lib.CP_ERR_UNSUPPORTED
+
+
 def test_permute_and_merge_reject_bad_arguments():
     L = lib()
     # Ulysses head limit: P must divide the head count
@@ -103,7 +108,7 @@ def test_permute_and_merge_reject_bad_arguments():
 
 
 # ------------------------------------------------------------ scheduler
-@pytest.mark.parametrize("layout", ["contiguous", "zigzag"])
+@pytest.mark.parametrize("layout", ["contiguous", "zigzag", "striped"])
 @pytest.mark.parametrize("P", [1, 2, 4, 8])
 @pytest.mark.parametrize("causal", [True, False])
 def test_schedule_matches_bruteforce(layout, P, causal):

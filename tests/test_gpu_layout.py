@@ -66,6 +66,22 @@ def test_zigzag_bit_exact(P, S, shape, dtype):
     assert np.array_equal(bits(z), bits(x))
 
 
+@pytest.mark.parametrize("P,S,shape,dtype", [
+    (4, 64, (8, 128), torch.bfloat16),
+    (8, 4096, (32, 128), torch.bfloat16),
+    (3, 36, (2, 5), torch.bfloat16),
+])
+def test_striped_bit_exact(P, S, shape, dtype):
+    x = synth.normal((S,) + shape, 6, 1.0, dtype).cuda()
+    y = api.striped_reorder(x, P)
+    assert np.array_equal(bits(y), np.take(bits(x), ref.striped_order(S, P), axis=0))
+    assert np.array_equal(bits(api.striped_reorder(y, P, inverse=True)), bits(x))
+    lse = synth.normal((4, S), 7, 1.0, torch.float32).cuda()
+    yl = api.striped_reorder(lse, P, seq_dim=1)
+    assert np.array_equal(bits(yl), np.take(bits(lse), ref.striped_order(S, P), axis=1))
+    assert torch.equal(api.striped_reorder(yl, P, inverse=True, seq_dim=1), lse)
+
+
 def test_zigzag_lse_rows():
     P, S, h = 8, 4096, 32
     lse = synth.normal((h, S), 9, 1.0, torch.float32).cuda()

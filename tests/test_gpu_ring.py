@@ -141,6 +141,31 @@ def test_full_size_ulysses_gqa_128k():
     compare(o[idx], lse[:, idx], want_o, want_l, what="full ulysses")
 
 
+# ----------------------------------------------------------- striped layout
+@pytest.mark.parametrize("P", [2, 4, 8])
+def test_striped_small(P):
+    ring_case(2048, 2, 1, 128, P, "striped")
+
+
+def test_striped_noncausal_dh64():
+    ring_case(1536, 4, 4, 64, 3, "striped", causal=False)
+
+
+def test_full_size_striped_64k():
+    S, P = 65536, 8
+    q, k, v = synth.qkv(S, 32, 32, 128)
+    qs, ks, vs = (api.striped_reorder(t.cuda(), P) for t in (q, k, v))
+    o, lse = api.ring_attn_fwd(qs, ks, vs, P, "striped", True)
+    o = api.striped_reorder(o, P, inverse=True)
+    lse = api.striped_reorder(lse, P, inverse=True, seq_dim=1)
+    torch.cuda.synchronize()
+    assert api.device_error() == 0
+    rows = sample_rows(S, P, "contiguous", n=128)
+    want_o, want_l = ref.attention(f64(q[torch.from_numpy(rows)]), f64(k), f64(v), causal=True, qpos=rows)
+    idx = torch.from_numpy(rows).cuda()
+    compare(o[idx], lse[:, idx], want_o, want_l, what="full striped")
+
+
 # ----------------------------------------------------------- more shapes
 @pytest.mark.parametrize("layout", ["contiguous", "zigzag"])
 def test_sixteen_ranks_split_launches(layout):

@@ -172,7 +172,7 @@ def test_matches_torch_sdpa_fp64_with_bool_mask():
 
 
 # ------------------------------------------------------------- invariants
-@pytest.mark.parametrize("layout", ["contiguous", "zigzag"])
+@pytest.mark.parametrize("layout", ["contiguous", "zigzag", "striped"])
 @pytest.mark.parametrize("P", [1, 2, 4])
 @pytest.mark.parametrize("causal", [True, False])
 def test_split_then_merge_equals_unsplit(layout, P, causal):
@@ -242,6 +242,21 @@ def test_merge_edge_cases():
 def test_zigzag_order_by_hand():
     # S=16, P=2: chunks of 4; rank 0 = chunks 0, 3; rank 1 = chunks 1, 2
     assert list(ref.zigzag_order(16, 2)) == [0, 1, 2, 3, 12, 13, 14, 15, 4, 5, 6, 7, 8, 9, 10, 11]
+
+
+def test_striped_order_by_hand():
+    # S=8, P=2: rank 0 holds even positions, rank 1 odd ones
+    assert list(ref.striped_order(8, 2)) == [0, 2, 4, 6, 1, 3, 5, 7]
+    assert sorted(ref.striped_order(48, 4)) == list(range(48))
+
+
+def test_striped_pairs_are_balanced_local_causal_blocks():
+    # every striped block pair is a local causal block: n(n+1)/2 admitted
+    # pairs for j <= r and n(n-1)/2 for j > r
+    S, P = 64, 4
+    n = S // P
+    for (r, t), (j, live, tot) in ref.pair_classes(S, P, "striped").items():
+        assert live == (n * (n + 1) // 2 if j <= r else n * (n - 1) // 2)
 
 
 def test_zigzag_round_trip_and_permutation():

@@ -8,8 +8,12 @@ already resident in HBM.  For the default workload (ring attention forward,
 S=32768, 32 heads, dh=128, P=4 contiguous causal shards, bf16) a step is the
 ring-step schedule, the block-attention launch over all live block pairs and
 the fp32 LSE merge, all through ``cp_ring_attn_fwd``; zigzag workloads add the
-zigzag reorder of Q, K, V and the inverse reorder of O and LSE; the Ulysses
-workload is seq->head transpose, per-group attention, head->seq transpose.
+zigzag (or striped) reorder of Q, K, V and the inverse reorder of O and LSE;
+the Ulysses workload is seq->head transpose, per-group attention, head->seq
+transpose; the hybrid workload (usp_gqa_128k) is the zigzag reorder over the
+ring groups, the seq->head transpose over the Ulysses ranks, the ring block
+pairs of every head block, a merge that writes the head blocks back, and the
+inverse reorder.
 
 The metric is causal-effective TFLOP/s (4 * dh * hq per admitted (q, k) pair,
 divided by the step time); the JSON line also carries the a2a-permute GB/s of
@@ -177,6 +181,22 @@ def make_workload(name, seq_len=None):
 
         def step():
             api.ulysses_attn_fwd(qd, kd, vd, P, True, o=o, lse=lse, workspace=ws)
+    elif layout == "usp":
+        Pr, Pu, rl = cfg["Pr"], cfg["Pu"], cfg["ring_layout"]
+        ws = torch.empty(api.usp_attn_workspace_size(S, hq, hkv, dh, Pr, Pu, rl, True), device=dev,
+                         dtype=torch.uint8)
+        qz, kz, vz = (torch.empty_like(t) for t in (qd, kd, vd))
+        oz = torch.empty_like(o)
+        lz = torch.empty_like(lse)
+        reorder = api.zigzag_reorder if rl == "zigzag" else api.striped_reorder
+
+        def step():
+            reorder(qd, Pr, out=qz)
+            reorder(kd, Pr, out=kz)
+            reorder(vd, Pr, out=vz)
+            api.usp_attn_fwd(qz, kz, vz, Pr, Pu, rl, True, o=oz, lse=lz, workspace=ws)
+            reorder(oz, Pr, inverse=True, out=o)
+            reorder(lz, Pr, inverse=True, seq_dim=1, out=lse)
     else:
         cu_dev = torch.tensor(cu, dtype=torch.int32, device=dev) if cu is not None else None
         ws = torch.empty(max(256, api.ring_attn_workspace_size(S, hq, hkv, dh, P, layout, True, dtype, cu)),
@@ -409,7 +429,8 @@ def run_ours(args, ws, rank, local):
                    "admitted_pairs": w["pairs"], "flops_per_step": w["flops"],
                    "l2": "inputs larger than L2 (Q+K+V %.0f MB, partials %.0f MB)" % (
                        sum(t.numel() * t.element_size() for t in w["in"]) / 1e6, w["ws_bytes"] / 1e6),
-                   "per_gpu": "independent problem per GPU"},
+                   "per_gpu": "independent problem per GPU",
+                   **({k_: cfg[k_] for k_ in ("Pr", "Pu", "ring_layout")} if w["layout"] == "usp" else {})},
         "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel", "achieved": attn_tf, "peak": pk["bf16"],
                      "unit": "TFLOP/s", "frac": attn_tf / pk["bf16"], "traffic": traffic,
                      "peak_source": pk["source"] + " burst bf16", "frac_of_sustained": attn_tf / pk["bf16_sus"],
@@ -437,7 +458,11 @@ def merge_bytes(w):
     """Algorithmic bytes of the merge: every live partial (O fp32 + LSE) read
     once, the output O and LSE written once."""
     from context_exact_attention_step_b200 import api
-    sch = api.ring_schedule(w["S"], w["P"], w["layout"], True, w["cu"])
+    cfg = w["cfg"]
+    if w["layout"] == "usp":  # Pu rings of Pr ranks over hq/Pu heads each
+        sch = api.ring_schedule(w["S"], cfg["Pr"], cfg["ring_layout"], True, w["cu"])
+    else:
+        sch = api.ring_schedule(w["S"], w["P"], w["layout"], True, w["cu"])
     rows = int(sch["q_rows"].sum())
     per_row = w["hq"] * (w["dh"] + 1) * 4
     return rows * per_row + w["S"] * per_row

@@ -1,6 +1,7 @@
 """B200 (sm_100a) context-parallel exact attention: ring-step block attention
-with partial (O, LSE), fp32 LSE merge, zigzag reorder and Ulysses
-sequence<->head transpose, with P virtual ranks on one GPU.
+with partial (O, LSE), fp32 LSE merge, zigzag and striped reorders, Ulysses
+sequence<->head transpose and the Ulysses-inside / Ring-across hybrid, with P
+virtual ranks on one GPU.
 
 The compute lives in ``libcp_attn.so`` (C ABI in ``include/cp_attn.h``);
 ``api`` is a thin PyTorch binding over it.
@@ -19,6 +20,8 @@ from .api import (  # noqa: F401
     ulysses_attn_fwd,
     ulysses_attn_workspace_size,
     ulysses_permute,
+    usp_attn_fwd,
+    usp_attn_workspace_size,
     zigzag_reorder,
 )
 

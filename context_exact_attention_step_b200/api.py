@@ -253,6 +253,42 @@ def ulysses_attn_fwd(q, k, v, P, causal=True, softmax_scale=0.0, o=None, lse=Non
     return o, lse
 
 
+def usp_attn_workspace_size(S, hq, hkv, dh, Pr, Pu, layout="contiguous", causal=True, cu_seqlens=None) -> int:
+    cu_p, n_docs, _keep = _cu_host(cu_seqlens)
+    out = ctypes.c_size_t(0)
+    check(lib().cp_usp_attn_workspace_size(S, hq, hkv, dh, Pr, Pu, _LAYOUTS[layout],
+                                           _lib.CP_MASK_CAUSAL if causal else _lib.CP_MASK_NONE, cu_p, n_docs,
+                                           ctypes.byref(out)))
+    return int(out.value)
+
+
+def usp_attn_fwd(q, k, v, Pr, Pu, layout="contiguous", causal=True, cu_seqlens=None, cu_seqlens_dev=None,
+                 softmax_scale=0.0, o=None, lse=None, workspace=None, stream=None):
+    """Ulysses inside groups of Pu virtual ranks, Ring across Pr groups.
+    q [S, hq, dh], k, v [S, hkv, dh] bf16 (CUDA) in the rank-major order of
+    ``layout`` over Pr ring shards (the buffer ring_attn_fwd takes with
+    P = Pr).  Returns (O [S, hq, dh] fp32, LSE [hq, S] fp32) in that order."""
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _need_cuda(n, t, torch.bfloat16)
+    S, hq, dh = q.shape
+    hkv = k.shape[1]
+    cu_p, n_docs, cu_np = _cu_host(cu_seqlens)
+    if n_docs > 0 and cu_seqlens_dev is None:
+        cu_seqlens_dev = torch.from_numpy(cu_np).to(q.device)
+    if o is None:
+        o = torch.empty((S, hq, dh), device=q.device, dtype=torch.float32)
+    if lse is None:
+        lse = torch.empty((hq, S), device=q.device, dtype=torch.float32)
+    if workspace is None:
+        need = usp_attn_workspace_size(S, hq, hkv, dh, Pr, Pu, layout, causal, cu_seqlens)
+        workspace = torch.empty(max(need, 256), device=q.device, dtype=torch.uint8)
+    check(lib().cp_usp_attn_fwd(_vp(q), _vp(k), _vp(v), S, hq, hkv, dh, Pr, Pu, _LAYOUTS[layout],
+                                _lib.CP_MASK_CAUSAL if causal else _lib.CP_MASK_NONE, cu_p, _vp(cu_seqlens_dev),
+                                n_docs, float(softmax_scale), _vp(o), _vp(lse), _vp(workspace), workspace.numel(),
+                                _stream(stream)))
+    return o, lse
+
+
 def ring_schedule(S, P, layout="contiguous", causal=True, cu_seqlens=None):
     """Host-only view of the ring-step schedule: arrays of P*P entries indexed
     r*P + t (see cp_ring_schedule)."""

@@ -218,11 +218,14 @@ struct Merge {
 };
 struct MergeTaskIn {
   int out_row0, rows;
+  int head_off = 0;
   std::vector<Merge> in;
 };
 
+// o_heads: heads per output row of O (h unless tasks scatter head blocks
+// into a wider output through head_off).
 cp_status run_merge(const std::vector<MergeTaskIn>& tasks, int h, int dh, float* o_out, float* lse_out,
-                    int lse_out_ld, void* o_bf16, cudaStream_t st) {
+                    int lse_out_ld, void* o_bf16, cudaStream_t st, int o_heads = 0) {
   static cp_merge_plan plan;
   static std::mutex mu;
   std::lock_guard<std::mutex> lk(mu);
@@ -232,6 +235,7 @@ cp_status run_merge(const std::vector<MergeTaskIn>& tasks, int h, int dh, float*
     plan.h = h;
     plan.dh = dh;
     plan.lse_out_ld = lse_out_ld;
+    plan.o_heads = o_heads > 0 ? o_heads : h;
     plan.o_out = o_out;
     plan.lse_out = lse_out;
     plan.o_out_bf16 = static_cast<uint16_t*>(o_bf16);
@@ -244,6 +248,7 @@ cp_status run_merge(const std::vector<MergeTaskIn>& tasks, int h, int dh, float*
       d.rows = t.rows;
       d.n_in = (int)t.in.size();
       d.in_begin = n_in;
+      d.head_off = t.head_off;
       for (const Merge& m : t.in) plan.inputs[n_in++] = {m.o, m.lse, m.row0, m.lse_ld};
       max_rows = std::max(max_rows, t.rows);
       ++i;
@@ -569,6 +574,125 @@ cp_status cp_ulysses_attn_fwd(const void* q, const void* k, const void* v, int S
   record(g_ev_attn_end, st);
   if ((e = launch_ulysses(oh, o, P, n, (size_t)hg * dh * 4, 1, st)) != cudaSuccess)
     return cuda_fail(e, "ulysses head->seq");
+  return ok();
+}
+
+static cp_status usp_check(int S, int hq, int hkv, int dh, int Pr, int Pu, cp_layout layout, cp_mask mask,
+                           const int32_t* cu_host, int n_docs) {
+  cp_status s;
+  if ((s = check_common(hq, hkv, dh)) != CP_OK) return s;
+  if (Pu < 1 || Pu > 64) return fail(CP_ERR_UNSUPPORTED, "Pu = %d (supported 1..64)", Pu);
+  if (hkv % Pu != 0) return fail(CP_ERR_UNSUPPORTED, "Pu (%d) must divide the KV head count (%d)", Pu, hkv);
+  if ((s = ring_check(S, hq / Pu, hkv / Pu, dh, Pr, layout, mask, CP_BF16, cu_host, n_docs)) != CP_OK) return s;
+  if (S % (Pr * Pu) != 0) return fail(CP_ERR_INVALID_ARG, "S = %d is not a multiple of Pr*Pu = %d", S, Pr * Pu);
+  if ((int64_t)Pu * S >= (1 << 30)) return fail(CP_ERR_UNSUPPORTED, "Pu * S = %lld rows", (long long)Pu * S);
+  return CP_OK;
+}
+
+// Workspace of the hybrid: head-major Q [Pu][S][hq/Pu][dh], K and V
+// [Pu][S][hkv/Pu][dh] (bf16), then Pu copies of the ring partials.
+static size_t usp_workspace(int S, int hq, int hkv, int dh, int Pu, const RingPlan& plan) {
+  return align256((size_t)S * hq * dh * 2) + 2 * align256((size_t)S * hkv * dh * 2) +
+         (size_t)Pu * align256(plan.partial_bytes);
+}
+
+cp_status cp_usp_attn_workspace_size(int S, int hq, int hkv, int dh, int Pr, int Pu, cp_layout layout, cp_mask mask,
+                                     const int32_t* cu_seqlens_host, int n_docs, size_t* bytes) {
+  cp_status s;
+  if (!bytes) return fail(CP_ERR_INVALID_ARG, "bytes is NULL");
+  if ((s = usp_check(S, hq, hkv, dh, Pr, Pu, layout, mask, cu_seqlens_host, n_docs)) != CP_OK) return s;
+  RingPlan plan = make_ring_plan(S, hq / Pu, dh, Pr, layout, mask, cu_seqlens_host, n_docs);
+  *bytes = usp_workspace(S, hq, hkv, dh, Pu, plan);
+  return ok();
+}
+
+cp_status cp_usp_attn_fwd(const void* q, const void* k, const void* v, int S, int hq, int hkv, int dh, int Pr, int Pu,
+                          cp_layout layout, cp_mask mask, const int32_t* cu_seqlens_host,
+                          const int32_t* cu_seqlens_dev, int n_docs, float softmax_scale, float* o, float* lse,
+                          void* workspace, size_t ws_bytes, void* stream) {
+  cp_status s;
+  if ((s = usp_check(S, hq, hkv, dh, Pr, Pu, layout, mask, cu_seqlens_host, n_docs)) != CP_OK) return s;
+  CP_CHECK_PTR(q);
+  CP_CHECK_PTR(k);
+  CP_CHECK_PTR(v);
+  CP_CHECK_PTR(o);
+  CP_CHECK_PTR(lse);
+  if (n_docs > 0 && !cu_seqlens_dev) return fail(CP_ERR_INVALID_ARG, "n_docs > 0 needs cu_seqlens_dev");
+  const int hg = hq / Pu, hkg = hkv / Pu;
+  RingPlan plan = make_ring_plan(S, hg, dh, Pr, layout, mask, cu_seqlens_host, n_docs);
+  const size_t need = usp_workspace(S, hq, hkv, dh, Pu, plan);
+  if (!workspace || ws_bytes < need)
+    return fail(CP_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws_bytes);
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return fail(CP_ERR_ALIGNMENT, "workspace is not 256-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  size_t off = 0;
+  void* qh = ws + off;
+  off += align256((size_t)S * hq * dh * 2);
+  void* kh = ws + off;
+  off += align256((size_t)S * hkv * dh * 2);
+  void* vh = ws + off;
+  off += align256((size_t)S * hkv * dh * 2);
+  uint8_t* parts = ws + off;
+  const size_t part_stride = align256(plan.partial_bytes);
+
+  // Ulysses seq->head inside every group at once: on one device the groups'
+  // sub-shards are consecutive rows, so the transpose over Pu with n = S/Pu
+  // gives head block u all S rows in storage order, out[u][row] = in[row][u].
+  cudaError_t e;
+  const int n = S / Pu;
+  if ((e = launch_ulysses(q, qh, Pu, n, (size_t)hg * dh * 2, 0, st)) != cudaSuccess ||
+      (e = launch_ulysses(k, kh, Pu, n, (size_t)hkg * dh * 2, 0, st)) != cudaSuccess ||
+      (e = launch_ulysses(v, vh, Pu, n, (size_t)hkg * dh * 2, 0, st)) != cudaSuccess)
+    return cuda_fail(e, "usp seq->head");
+
+  // Ring across the groups for every head block: head block u's rows start
+  // at u*S in the head-major buffers.  Pairs keep the heaviest-first order of
+  // the ring plan, head blocks interleaved.
+  std::vector<PairIn> pairs;
+  pairs.reserve(plan.pairs.size() * Pu);
+  for (const PairPlan& pp : plan.pairs)
+    for (int u = 0; u < Pu; ++u) {
+      PairIn pi;
+      pi.q = pp.q;
+      pi.k = pp.k;
+      for (Seg& x : pi.q) x.buf_row += u * S;
+      for (Seg& x : pi.k) x.buf_row += u * S;
+      pi.qtiles = pp.qtiles;
+      uint8_t* pu = parts + (size_t)u * part_stride;
+      pi.o = reinterpret_cast<float*>(pu + pp.o_off);
+      pi.lse = reinterpret_cast<float*>(pu + pp.lse_off);
+      pi.lse_ld = pp.rows;
+      pi.reverse = mask == CP_MASK_CAUSAL;
+      pairs.push_back(std::move(pi));
+    }
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)dh);
+  record(g_ev_attn_begin, st);
+  if ((s = run_pairs(qh, kh, vh, (int64_t)Pu * S, (int64_t)Pu * S, hg, hkg, dh, mask == CP_MASK_CAUSAL,
+                     cu_seqlens_dev, n_docs, scale, pairs, st)) != CP_OK)
+    return s;
+  record(g_ev_attn_end, st);
+
+  // Merge per head block, writing heads [u*hg, (u+1)*hg) of every output
+  // row: the head->seq transpose happens in the merge's stores.
+  std::vector<MergeTaskIn> tasks;
+  for (int u = 0; u < Pu; ++u) {
+    const uint8_t* pu = parts + (size_t)u * part_stride;
+    for (const MergeTaskPlan& tp : plan.tasks) {
+      MergeTaskIn t;
+      t.out_row0 = tp.row0;
+      t.rows = tp.rows;
+      t.head_off = u * hg;
+      for (const auto& in : tp.inputs) {
+        const PairPlan& pp = plan.pairs[in.first];
+        t.in.push_back({reinterpret_cast<const float*>(pu + pp.o_off),
+                        reinterpret_cast<const float*>(pu + pp.lse_off), in.second, pp.rows});
+      }
+      tasks.push_back(std::move(t));
+    }
+  }
+  if ((s = run_merge(tasks, hg, dh, o, lse, S, nullptr, st, hq)) != CP_OK) return s;
+  record(g_ev_merge_end, st);
   return ok();
 }
 

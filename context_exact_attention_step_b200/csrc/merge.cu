@@ -90,18 +90,20 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(const __grid_constant__ 
   acc.z *= inv;
   acc.w *= inv;
   const size_t orow = (size_t)(task.out_row0 + row);
-  __stcs(reinterpret_cast<float4*>(plan.o_out + (orow * h + head) * DH) + sub, acc);
+  const size_t ohead = (size_t)task.head_off + head;
+  const size_t oidx = (orow * plan.o_heads + ohead) * DH;
+  __stcs(reinterpret_cast<float4*>(plan.o_out + oidx) + sub, acc);
   if (plan.o_out_bf16) {
     const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
     const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
     uint2 pk;
     pk.x = *reinterpret_cast<const uint32_t*>(&lo);
     pk.y = *reinterpret_cast<const uint32_t*>(&hi);
-    reinterpret_cast<uint2*>(plan.o_out_bf16 + (orow * h + head) * DH)[sub] = pk;
+    reinterpret_cast<uint2*>(plan.o_out_bf16 + oidx)[sub] = pk;
   }
   if (sub == 0) {
     const float lse = tot > 0.f ? m + logf(tot) : -CUDART_INF_F;
-    plan.lse_out[(size_t)head * plan.lse_out_ld + orow] = lse;
+    plan.lse_out[ohead * plan.lse_out_ld + orow] = lse;
   }
 }
 

@@ -52,7 +52,9 @@ struct cp_attn_plan {
 
 // Merge: rows [out_row0, out_row0 + rows) of the output are the LSE-weighted
 // fold of n_in partial results; input i supplies row (row0 + x) for output
-// row (out_row0 + x).
+// row (out_row0 + x).  A task covers h heads of its inputs and writes them as
+// heads [head_off, head_off + h) of an output whose rows hold o_heads heads,
+// so a merge can scatter head blocks straight into a wider output.
 struct cp_merge_input {
   const float* o;      // [.][h][dh]
   const float* lse;    // [h][lse_ld]
@@ -65,14 +67,16 @@ struct cp_merge_task {
   int32_t rows;
   int32_t n_in;
   int32_t in_begin;
+  int32_t head_off;      // first output head of the task's h heads
 };
 
 struct cp_merge_plan {
   int32_t n_tasks;
   int32_t h, dh;
   int32_t lse_out_ld;
-  float* o_out;          // [.][h][dh]
-  float* lse_out;        // [h][lse_out_ld]
+  int32_t o_heads;       // heads per output row of O (>= head_off + h)
+  float* o_out;          // [.][o_heads][dh]
+  float* lse_out;        // [o_heads][lse_out_ld]
   uint16_t* o_out_bf16;  // optional bf16 copy of O (nullable)
   cp_merge_task tasks[CP_MAX_TASKS];
   cp_merge_input inputs[CP_MAX_INPUTS];

@@ -58,7 +58,7 @@ def cu_seqlens_from_lengths(lens):
     return torch.tensor(cu, dtype=torch.int32)
 
 
-# The five workloads the library is measured on.
+# The workloads the library is tested and measured on.
 CONFIGS = {
     "tiny_ring_fp32": dict(S=1024, hq=4, hkv=4, dh=64, P=4, layout="contiguous",
                            causal=True, varlen=False, std=1.0, dtype="fp32"),
@@ -70,6 +70,10 @@ CONFIGS = {
                              causal=True, varlen=False, std=0.5, dtype="bf16"),
     "ulysses_gqa_128k": dict(S=131072, hq=32, hkv=8, dh=128, P=8, layout="ulysses",
                              causal=True, varlen=False, std=0.5, dtype="bf16"),
+    # Ulysses over Pu = 4 ranks inside each of Pr = 2 zigzag ring groups: 8
+    # ranks against 4 KV heads, which Ulysses alone cannot shard.
+    "usp_gqa_128k": dict(S=131072, hq=32, hkv=4, dh=128, P=8, Pr=2, Pu=4, layout="usp", ring_layout="zigzag",
+                         causal=True, varlen=False, std=0.5, dtype="bf16"),
     "varlen_zigzag_128k": dict(S=131072, hq=32, hkv=32, dh=128, P=8, layout="zigzag",
                                causal=True, varlen=True, std=0.5, dtype="bf16",
                                doc_lo=1024, doc_hi=32768),

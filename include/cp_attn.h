@@ -218,6 +218,43 @@ cp_status cp_ulysses_attn_fwd(const void* q, const void* k, const void* v, int S
                               size_t ws_bytes, void* stream);
 
 /*
+ * cp_usp_attn_workspace_size / cp_usp_attn_fwd -- the two-dimensional hybrid
+ * of the two methods: P = Pr * Pu virtual ranks, DeepSpeed-Ulysses inside
+ * each group of Pu ranks and Ring Attention across the Pr groups ("序列並行"
+ * concept page (compassingai), closing section: Ulysses all-to-all inside the
+ * NVLink domain, Ring P2P across it, which lifts the head-count limit;
+ * "Context Parallelism" write-up (pwwt.cn) §6: Ulysses head regrouping inside
+ * the CP group, then the Ring passes the sequence).
+ *
+ * Layout: group g is ring shard g of `layout` over Pr ranks (contiguous,
+ * zigzag or striped, exactly the rank-major buffer cp_ring_attn_fwd takes
+ * with P = Pr); its S/Pr rows are split into Pu consecutive sub-shards, sub-
+ * rank u of group g being rank g*Pu + u.  Inputs q [S][hq][dh], k, v
+ * [S][hkv][dh] bf16 in that storage order; outputs o [S][hq][dh] fp32 and
+ * lse [hq][S] fp32 in the same order (row i of o is row i of q).
+ *
+ * Steps: Ulysses seq->head transpose of Q, K, V over Pu (every group at
+ * once); one attention launch for every live ring block pair of every head
+ * block (the ring schedule of cp_ring_attn_fwd with P = Pr); one merge launch
+ * that folds each head block's partials and writes them directly as heads
+ * [u*hq/Pu, (u+1)*hq/Pu) of o and lse, which is the head->seq transpose.
+ *
+ * Workspace (caller-owned, 256-byte aligned, size from
+ * cp_usp_attn_workspace_size with the same arguments): head-major bf16 copies
+ * of Q, K, V plus Pu sets of ring partials.
+ * Supported: Pu | hkv (KV heads are not replicated), 1 <= Pr <= 16,
+ * S % (Pr*Pu) == 0 (and S % (2*Pr) == 0 for zigzag), dh in {64, 128}; documents
+ * (cu_seqlens, as for cp_ring_attn_fwd) with the contiguous and zigzag
+ * layouts.  Errors as for cp_ring_attn_fwd; nothing is launched on error.
+ */
+cp_status cp_usp_attn_workspace_size(int S, int hq, int hkv, int dh, int Pr, int Pu, cp_layout layout, cp_mask mask,
+                                     const int32_t* cu_seqlens_host, int n_docs, size_t* bytes);
+cp_status cp_usp_attn_fwd(const void* q, const void* k, const void* v, int S, int hq, int hkv, int dh, int Pr, int Pu,
+                          cp_layout layout, cp_mask mask, const int32_t* cu_seqlens_host,
+                          const int32_t* cu_seqlens_dev, int n_docs, float softmax_scale, float* o, float* lse,
+                          void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * Host-only inspection of the ring-step schedule (no GPU needed).  For every
  * rank r and step t (index r*P + t):
  *   src[r*P+t]        the key/value shard j = (r - t) mod P held at that step

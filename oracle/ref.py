@@ -29,6 +29,8 @@ definition itself:
 * ``ulysses_seq_to_head`` / ``ulysses_head_to_seq`` -- the all-to-all
   transpose [S/P, H, d_h] -> [S, H/P, d_h] (compassingai §三 "Ulysses 的
   AllToAll 轉置"; pwwt.cn §2.3), device i taking head block i.
+* ``usp_attention``      -- the Ulysses-inside / Ring-across hybrid, composed
+  from the functions above (compassingai, closing section; pwwt.cn §6).
 * ``live_pair_count``    -- number of (q, k) pairs the explicit mask admits
   (brute force), the unit of the causal-effective FLOP count.
 """
@@ -240,6 +242,59 @@ def ring_attention(q, k, v, S, P, layout, causal=True, cu_seqlens=None, scale=No
         outs.append(o_r)
         lses.append(l_r)
     return np.concatenate(outs, axis=0), np.concatenate(lses, axis=1)
+
+
+def usp_attention(q, k, v, S, Pr, Pu, layout, causal=True, cu_seqlens=None, scale=None):
+    """USP, the two-dimensional hybrid: P = Pr * Pu ranks, Ulysses inside each
+    group of Pu ranks and Ring across the Pr groups ("序列並行（Sequence
+    Parallelism）" concept page (compassingai), closing section on mixing the
+    two: Ulysses all-to-all inside the NVLink domain, Ring P2P across it;
+    "Context Parallelism" write-up (pwwt.cn) §2 comparison and §6: first the
+    Ulysses head regrouping inside the CP group, then the Ring passes the
+    sequence).
+
+    Reading taken: group g is ring shard g of ``layout`` over Pr ranks; its
+    m = S/Pr tokens are split into Pu consecutive sub-shards of n = m/Pu tokens,
+    sub-rank u of group g being global rank g*Pu + u.  Steps:
+      1. Ulysses seq->head inside each group: sub-rank u gathers all m tokens of
+         its group for query heads [u*Hq/Pu, ...) and KV heads [u*Hkv/Pu, ...);
+      2. for each head block u, a ring over the Pr groups: group g holds KV
+         shard j = (g - t) mod Pr at step t, the partials are folded by
+         ``lse_merge``;
+      3. Ulysses head->seq inside each group.
+    Inputs in natural order [S, H, dh]; outputs in the storage order of the
+    ranks (the ring layout over Pr, rank-major): O [S, Hq, dh], LSE [Hq, S]."""
+    q = np.asarray(q)
+    k = np.asarray(k)
+    v = np.asarray(v)
+    hq, hkv, dh = q.shape[1], k.shape[1], q.shape[2]
+    assert hq % Pu == 0 and hkv % Pu == 0 and S % (Pr * Pu) == 0
+    m = S // Pr
+    n = m // Pu
+    hg = hq // Pu
+    pos = [shard_positions(S, Pr, layout, g) for g in range(Pr)]
+    # step 1: per group, [Pu, n, H, dh] -> [Pu, m, H/Pu, dh]
+    qh = [ulysses_seq_to_head(q[pos[g]].reshape(Pu, n, hq, dh), Pu) for g in range(Pr)]
+    kh = [ulysses_seq_to_head(k[pos[g]].reshape(Pu, n, hkv, dh), Pu) for g in range(Pr)]
+    vh = [ulysses_seq_to_head(v[pos[g]].reshape(Pu, n, hkv, dh), Pu) for g in range(Pr)]
+    # step 2: ring across groups, one per head block
+    o_grp = [np.zeros((Pu, m, hg, dh)) for _ in range(Pr)]
+    lse_grp = [np.zeros((Pu, hg, m)) for _ in range(Pr)]
+    for u in range(Pu):
+        for g in range(Pr):
+            parts_o, parts_l = [], []
+            for t in range(Pr):
+                j = ring_source(g, t, Pr)
+                o_p, l_p = attention(qh[g][u], kh[j][u], vh[j][u], causal=causal, cu_seqlens=cu_seqlens,
+                                     scale=scale, qpos=pos[g], kpos=pos[j])
+                parts_o.append(o_p)
+                parts_l.append(l_p)
+            o_grp[g][u], lse_grp[g][u] = lse_merge(np.stack(parts_o), np.stack(parts_l))
+    # step 3: per group, [Pu, m, H/Pu, dh] -> [Pu, n, H, dh]; LSE head block u
+    # of group g covers heads [u*hg, (u+1)*hg) and the group's m rows
+    o = np.concatenate([ulysses_head_to_seq(o_grp[g], Pu).reshape(m, hq, dh) for g in range(Pr)], axis=0)
+    lse = np.concatenate([lse_grp[g].reshape(hq, m) for g in range(Pr)], axis=1)
+    return o, lse
 
 
 def live_pair_count(S, causal=True, cu_seqlens=None, qpos=None, kpos=None):

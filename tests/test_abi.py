@@ -92,6 +92,37 @@ def test_striped_rejects_documents():
     assert _ring(layout=_lib.CP_LAYOUT_STRIPED, cu=cu, n_docs=2) == _lib.CP_ERR_UNSUPPORTED
 
 
+def _usp(S=1024, hq=8, hkv=4, dh=128, Pr=2, Pu=2, layout=_lib.CP_LAYOUT_ZIGZAG, cu=None, n_docs=0, ws=FAKE,
+         wsb=1 << 40):
+    return lib().cp_usp_attn_fwd(FAKE, FAKE, FAKE, S, hq, hkv, dh, Pr, Pu, layout, _lib.CP_MASK_CAUSAL, cu,
+                                 ctypes.c_void_p(0) if not n_docs else FAKE, n_docs, 0.0, FAKE, FAKE, ws, wsb,
+                                 ctypes.c_void_p(0))
+
+
+def test_usp_rejects_bad_arguments():
+    assert _usp(hkv=4, Pu=8, hq=8) == _lib.CP_ERR_UNSUPPORTED        # Pu does not divide the KV heads
+    assert _usp(S=1026, Pr=2, Pu=2, layout=_lib.CP_LAYOUT_CONTIGUOUS) == _lib.CP_ERR_INVALID_ARG  # Pr*Pu
+    assert _usp(S=1026, Pr=2, Pu=1) == _lib.CP_ERR_INVALID_ARG        # 2*Pr does not divide S (zigzag)
+    assert _usp(Pr=17) == _lib.CP_ERR_UNSUPPORTED
+    assert _usp(dh=96) == _lib.CP_ERR_UNSUPPORTED
+    assert _usp(ws=ctypes.c_void_p(0), wsb=0) == _lib.CP_ERR_WORKSPACE
+    assert _usp(wsb=1024) == _lib.CP_ERR_WORKSPACE
+    cu = (ctypes.c_int32 * 3)(0, 600, 1024)
+    assert _usp(layout=_lib.CP_LAYOUT_STRIPED, cu=cu, n_docs=2) == _lib.CP_ERR_UNSUPPORTED
+    assert len(lib().cp_last_error_string()) > 0
+
+
+@pytest.mark.parametrize("layout", ["contiguous", "zigzag", "striped"])
+def test_usp_workspace_is_copies_plus_pu_rings(layout):
+    # head-major bf16 Q, K, V, then one set of ring partials (P = Pr, hq/Pu
+    # heads) per Ulysses head block
+    S, hq, hkv, dh, Pr, Pu = 4096, 32, 4, 128, 2, 4
+    ring = api.ring_attn_workspace_size(S, hq // Pu, hkv // Pu, dh, Pr, layout)
+    a = lambda x: (x + 255) // 256 * 256
+    want = a(S * hq * dh * 2) + 2 * a(S * hkv * dh * 2) + Pu * a(ring)
+    assert api.usp_attn_workspace_size(S, hq, hkv, dh, Pr, Pu, layout) == want
+
+
 def test_permute_and_merge_reject_bad_arguments():
     L = lib()
     # Ulysses head limit: P must divide the head count

@@ -299,6 +299,56 @@ def test_ulysses_composite_equals_attention():
     np.testing.assert_allclose(back, o, atol=1e-12)
 
 
+def _storage_order(S, P, layout):
+    return np.concatenate([ref.shard_positions(S, P, layout, r) for r in range(P)])
+
+
+@pytest.mark.parametrize("layout", ["contiguous", "zigzag", "striped"])
+@pytest.mark.parametrize("Pr,Pu", [(2, 2), (4, 2), (2, 4), (1, 4), (3, 2)])
+@pytest.mark.parametrize("causal", [True, False])
+def test_usp_equals_unsplit_attention(layout, Pr, Pu, causal):
+    # The hybrid is exact (compassingai §二: the block recurrence loses
+    # nothing), so in storage order it must equal attention of the whole
+    # sequence.  GQA 8:4, so each Ulysses head block has its own KV heads.
+    S, Hq, Hkv, dh = 48, 8, 4, 8
+    q, k, v = randn(S, Hq, dh), randn(S, Hkv, dh), randn(S, Hkv, dh)
+    o, lse = ref.attention(q, k, v, causal=causal)
+    o_u, lse_u = ref.usp_attention(q, k, v, S, Pr, Pu, layout, causal=causal)
+    order = _storage_order(S, Pr, layout)
+    np.testing.assert_allclose(o_u, o[order], atol=1e-12)
+    np.testing.assert_allclose(lse_u, lse[:, order], atol=1e-12)
+
+
+def test_usp_with_documents_equals_unsplit():
+    S, Hq, Hkv, dh, Pr, Pu = 64, 4, 2, 8, 2, 2
+    cu = [0, 5, 6, 41, 64]
+    q, k, v = randn(S, Hq, dh), randn(S, Hkv, dh), randn(S, Hkv, dh)
+    o, lse = ref.attention(q, k, v, causal=True, cu_seqlens=cu)
+    o_u, lse_u = ref.usp_attention(q, k, v, S, Pr, Pu, "zigzag", causal=True, cu_seqlens=cu)
+    order = _storage_order(S, Pr, "zigzag")
+    np.testing.assert_allclose(o_u, o[order], atol=1e-12)
+    np.testing.assert_allclose(lse_u, lse[:, order], atol=1e-12)
+
+
+def test_usp_special_cases_reduce_to_ring_and_ulysses():
+    S, Hq, Hkv, dh = 32, 4, 2, 8
+    q, k, v = randn(S, Hq, dh), randn(S, Hkv, dh), randn(S, Hkv, dh)
+    # Pu = 1: no Ulysses dimension, the hybrid is the plain ring over Pr ranks
+    o_u, l_u = ref.usp_attention(q, k, v, S, 4, 1, "zigzag")
+    o_r, l_r = ref.ring_attention(q, k, v, S, 4, "zigzag")
+    np.testing.assert_allclose(o_u, o_r, atol=1e-12)
+    np.testing.assert_allclose(l_u, l_r, atol=1e-12)
+    # Pr = 1: no ring dimension, the hybrid is Ulysses over Pu ranks
+    P = 2
+    n = S // P
+    qh = ref.ulysses_seq_to_head(q.reshape(P, n, Hq, dh), P)
+    kh = ref.ulysses_seq_to_head(k.reshape(P, n, Hkv, dh), P)
+    vh = ref.ulysses_seq_to_head(v.reshape(P, n, Hkv, dh), P)
+    oh = np.stack([ref.attention(qh[r], kh[r], vh[r], causal=True)[0] for r in range(P)])
+    o_u, _ = ref.usp_attention(q, k, v, S, 1, P, "contiguous")
+    np.testing.assert_allclose(o_u, ref.ulysses_head_to_seq(oh, P).reshape(S, Hq, dh), atol=1e-12)
+
+
 # ------------------------------------------------------ work counts
 def test_live_pair_counts_closed_forms():
     S = 96

@@ -31,6 +31,10 @@ definition itself:
   AllToAll 轉置"; pwwt.cn §2.3), device i taking head block i.
 * ``usp_attention``      -- the Ulysses-inside / Ring-across hybrid, composed
   from the functions above (compassingai, closing section; pwwt.cn §6).
+* ``attention_bwd`` / ``ring_attention_bwd`` -- the gradient of the exact
+  attention for an upstream dO: by definition over the whole score matrix, and
+  the ring form (per block pair with the merged LSE, KV gradients travelling
+  with their shard).
 * ``live_pair_count``    -- number of (q, k) pairs the explicit mask admits
   (brute force), the unit of the causal-effective FLOP count.
 """
@@ -295,6 +299,101 @@ def usp_attention(q, k, v, S, Pr, Pu, layout, causal=True, cu_seqlens=None, scal
     o = np.concatenate([ulysses_head_to_seq(o_grp[g], Pu).reshape(m, hq, dh) for g in range(Pr)], axis=0)
     lse = np.concatenate([lse_grp[g].reshape(hq, m) for g in range(Pr)], axis=1)
     return o, lse
+
+
+# --------------------------------------------------------------------------
+# backward
+# --------------------------------------------------------------------------
+def attention_bwd(q, k, v, do, causal=True, cu_seqlens=None, scale=None, qpos=None, kpos=None,
+                  row_block=256):
+    """Gradients of ``attention``'s O with respect to q, k, v for an upstream
+    gradient ``do`` [Sq, Hq, dh], in float64, from the definition of the
+    masked softmax: with P the attention probabilities (explicit mask, every
+    key at once),
+        dV = P^T dO,  dP = dO V^T,  dS = P * (dP - rowsum(P * dP)),
+        dQ = scale * dS K,  dK = scale * dS^T Q,
+    where GQA sums dK, dV over the query heads that share a KV head.  The
+    pages state no backward; this is the gradient of the exact attention they
+    define (training runs both passes: the DeepSpeed-Ulysses / ring-flash-
+    attention how-to (2kiu.com), §4 "启动命令与显存吞吐验证", checks memory
+    after the forward and after the backward).  Returns dQ [Sq, Hq, dh],
+    dK, dV [Sk, Hkv, dh]."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    do = np.asarray(do, dtype=np.float64)
+    sq, hq, dh = q.shape
+    sk, hkv, _ = k.shape
+    group = hq // hkv
+    if scale is None:
+        scale = 1.0 / math.sqrt(dh)
+    qpos = np.arange(sq) if qpos is None else np.asarray(qpos)
+    kpos = np.arange(sk) if kpos is None else np.asarray(kpos)
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for r0 in range(0, sq, row_block):
+        r1 = min(sq, r0 + row_block)
+        mask = explicit_mask(qpos[r0:r1], kpos, causal, cu_seqlens)
+        live = mask.any(axis=1)
+        for h in range(hq):
+            g = h // group
+            s = np.where(mask, (q[r0:r1, h, :] @ k[:, g, :].T) * scale, NEG_INF)
+            m = np.where(live, np.max(s, axis=1, initial=NEG_INF), 0.0)
+            e = np.where(mask, np.exp(s - m[:, None]), 0.0)
+            l = np.where(live, e.sum(axis=1), 1.0)
+            p = e / l[:, None]
+            dp = do[r0:r1, h, :] @ v[:, g, :].T
+            ds = p * (dp - (p * dp).sum(axis=1, keepdims=True))
+            dv[:, g, :] += p.T @ do[r0:r1, h, :]
+            dq[r0:r1, h, :] = scale * (ds @ k[:, g, :])
+            dk[:, g, :] += scale * (ds.T @ q[r0:r1, h, :])
+    return dq, dk, dv
+
+
+def ring_attention_bwd(q, k, v, do, S, P, layout, causal=True, cu_seqlens=None, scale=None):
+    """Ring backward over P virtual ranks: the forward's merged O and LSE of
+    each rank are kept; at ring step t rank r holds KV shard j = (r - t) mod P
+    and, with P_rj = exp(scale Q_r K_j^T - LSE_r) (the merged LSE, so P_rj is
+    the true slice of the global probabilities) and D_r = rowsum(dO_r * O_r),
+        dS_rj = P_rj * (dO_r V_j^T - D_r),
+        dQ_r += scale dS_rj K_j,  dK_j += scale dS_rj^T Q_r,  dV_j += P_rj^T dO_r,
+    the KV gradients travelling with their shard.  Inputs q, k, v, do in
+    natural order; outputs in rank-major storage order (dQ [S, Hq, dh],
+    dK, dV [S, Hkv, dh])."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    do = np.asarray(do, dtype=np.float64)
+    hq, dh = q.shape[1], q.shape[2]
+    hkv = k.shape[1]
+    group = hq // hkv
+    if scale is None:
+        scale = 1.0 / math.sqrt(dh)
+    o_all, lse_all = ring_attention(q, k, v, S, P, layout, causal, cu_seqlens, scale)
+    pos = [shard_positions(S, P, layout, r) for r in range(P)]
+    n = pos[0].size
+    dq = [np.zeros((n, hq, dh)) for _ in range(P)]
+    dk = [np.zeros((n, hkv, dh)) for _ in range(P)]
+    dv = [np.zeros((n, hkv, dh)) for _ in range(P)]
+    for t in range(P):
+        for r in range(P):
+            j = ring_source(r, t, P)
+            qp, kp = pos[r], pos[j]
+            o_r = o_all[r * n:(r + 1) * n]
+            lse_r = lse_all[:, r * n:(r + 1) * n]
+            mask = explicit_mask(qp, kp, causal, cu_seqlens)
+            for h in range(hq):
+                g = h // group
+                s = (q[qp, h, :] @ k[kp, g, :].T) * scale
+                lse_h = np.where(np.isfinite(lse_r[h]), lse_r[h], 0.0)
+                p = np.where(mask, np.exp(s - lse_h[:, None]), 0.0)
+                d = (do[qp, h, :] * o_r[:, h, :]).sum(axis=1)
+                ds = p * (do[qp, h, :] @ v[kp, g, :].T - d[:, None])
+                dq[r][:, h, :] += scale * (ds @ k[kp, g, :])
+                dk[j][:, g, :] += scale * (ds.T @ q[qp, h, :])
+                dv[j][:, g, :] += p.T @ do[qp, h, :]
+    return np.concatenate(dq), np.concatenate(dk), np.concatenate(dv)
 
 
 def live_pair_count(S, causal=True, cu_seqlens=None, qpos=None, kpos=None):

@@ -349,6 +349,101 @@ def test_usp_special_cases_reduce_to_ring_and_ulysses():
     np.testing.assert_allclose(o_u, ref.ulysses_head_to_seq(oh, P).reshape(S, Hq, dh), atol=1e-12)
 
 
+# ------------------------------------------------------ backward
+def _torch_grads(q, k, v, do, causal, cu=None, scale=None):
+    """Gradients by torch autograd (fp64, CPU) of masked softmax attention
+    written with plain torch ops and an explicit boolean mask."""
+    S, hq, dh = q.shape
+    hkv = k.shape[1]
+    scale = 1.0 / math.sqrt(dh) if scale is None else scale
+    tq, tk, tv = (torch.tensor(x, dtype=torch.float64, requires_grad=True) for x in (q, k, v))
+    mask = torch.from_numpy(ref.explicit_mask(np.arange(S), np.arange(k.shape[0]), causal, cu))
+    kk = tk.repeat_interleave(hq // hkv, dim=1)
+    vv = tv.repeat_interleave(hq // hkv, dim=1)
+    s = torch.einsum("qhd,khd->hqk", tq, kk) * scale
+    s = s.masked_fill(~mask[None], float("-inf"))
+    o = torch.einsum("hqk,khd->qhd", torch.softmax(s, dim=-1), vv)
+    o.backward(torch.tensor(do, dtype=torch.float64))
+    return tq.grad.numpy(), tk.grad.numpy(), tv.grad.numpy()
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_bwd_matches_torch_autograd(causal):
+    S, hq, hkv, dh = 40, 4, 2, 8
+    q, k, v, do = randn(S, hq, dh), randn(S, hkv, dh), randn(S, hkv, dh), randn(S, hq, dh)
+    cu = [0, 9, 10, 40]
+    for docs in (None, cu):
+        got = ref.attention_bwd(q, k, v, do, causal=causal, cu_seqlens=docs)
+        want = _torch_grads(q, k, v, do, causal, docs)
+        for g, w in zip(got, want):
+            np.testing.assert_allclose(g, w, atol=1e-12)
+
+
+def test_bwd_matches_finite_differences():
+    # central differences of L = sum(dO * O) on a tiny causal GQA case
+    S, hq, hkv, dh = 6, 2, 1, 3
+    q, k, v, do = randn(S, hq, dh), randn(S, hkv, dh), randn(S, hkv, dh), randn(S, hq, dh)
+    dq, dk, dv = ref.attention_bwd(q, k, v, do, causal=True)
+    loss = lambda a, b, c: float((ref.attention(a, b, c, causal=True)[0] * do).sum())
+    eps = 1e-6
+    for x, g, idx in ((q, dq, 0), (k, dk, 1), (v, dv, 2)):
+        num = np.zeros_like(x)
+        for i in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[i] += eps
+            xm[i] -= eps
+            args_p = [q, k, v]
+            args_m = [q, k, v]
+            args_p[idx], args_m[idx] = xp, xm
+            num[i] = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+        np.testing.assert_allclose(g, num, atol=1e-7)
+
+
+def test_bwd_closed_forms_and_invariants():
+    S, hq, hkv, dh = 32, 4, 2, 8
+    q, k, v, do = randn(S, hq, dh), randn(S, hkv, dh), randn(S, hkv, dh), randn(S, hq, dh)
+    dq, dk, dv = ref.attention_bwd(q, k, v, do, causal=True)
+    # every row of dS sums to zero, so the key gradients of a KV head sum to 0
+    np.testing.assert_allclose(dk.sum(axis=0), 0.0, atol=1e-10)
+    # every row of P sums to one, so the value gradients of a KV head sum to
+    # the upstream gradients of its query heads
+    want = do.reshape(S, hkv, hq // hkv, dh).sum(axis=(0, 2))
+    np.testing.assert_allclose(dv.sum(axis=0), want, atol=1e-10)
+    # causal row 0 sees only key 0: its softmax is constant, so dQ_0 = 0
+    np.testing.assert_allclose(dq[0], 0.0, atol=1e-12)
+    # identical keys: P is uniform over the live keys whatever q is, so dQ = 0
+    k1 = np.repeat(randn(1, hkv, dh), S, axis=0)
+    dq1, _, _ = ref.attention_bwd(q, k1, v, do, causal=True)
+    np.testing.assert_allclose(dq1, 0.0, atol=1e-12)
+
+
+@pytest.mark.parametrize("layout", ["contiguous", "zigzag", "striped"])
+@pytest.mark.parametrize("P", [1, 2, 4])
+@pytest.mark.parametrize("causal", [True, False])
+def test_ring_bwd_equals_unsplit(layout, P, causal):
+    # the ring form with the merged LSE is exact: it equals the gradient of
+    # the unsplit attention, in storage order
+    S, hq, hkv, dh = 32, 4, 2, 8
+    q, k, v, do = randn(S, hq, dh), randn(S, hkv, dh), randn(S, hkv, dh), randn(S, hq, dh)
+    dq, dk, dv = ref.attention_bwd(q, k, v, do, causal=causal)
+    rq, rk, rv = ref.ring_attention_bwd(q, k, v, do, S, P, layout, causal=causal)
+    order = _storage_order(S, P, layout)
+    np.testing.assert_allclose(rq, dq[order], atol=1e-12)
+    np.testing.assert_allclose(rk, dk[order], atol=1e-12)
+    np.testing.assert_allclose(rv, dv[order], atol=1e-12)
+
+
+def test_ring_bwd_with_documents_equals_unsplit():
+    S, hq, hkv, dh, P = 64, 2, 2, 8, 4
+    cu = [0, 3, 30, 31, 64]
+    q, k, v, do = randn(S, hq, dh), randn(S, hkv, dh), randn(S, hkv, dh), randn(S, hq, dh)
+    dq, dk, dv = ref.attention_bwd(q, k, v, do, causal=True, cu_seqlens=cu)
+    rq, rk, rv = ref.ring_attention_bwd(q, k, v, do, S, P, "zigzag", causal=True, cu_seqlens=cu)
+    order = _storage_order(S, P, "zigzag")
+    for a, b in ((rq, dq), (rk, dk), (rv, dv)):
+        np.testing.assert_allclose(a, b[order], atol=1e-12)
+
+
 # ------------------------------------------------------ work counts
 def test_live_pair_counts_closed_forms():
     S = 96
@@ -401,3 +496,36 @@ def test_pins_catch_planted_mistakes(monkeypatch):
     q2, k2 = randn(S, H, dh), randn(S, H, dh)
     _, lse_bad = ref.attention(q2, k2, v, causal=True, scale=1.0 / dh)
     assert abs(lse_bad[0, 0] - float(q2[0, 0] @ k2[0, 0]) / 2.0) > 1e-6
+
+
+def test_bwd_pins_catch_planted_mistakes(monkeypatch):
+    """A dropped D term (dS = P * dP) and a transposed GQA sum in the ring
+    backward are each caught by a pin above."""
+    S, hq, hkv, dh = 16, 2, 1, 4
+    q, k, v, do = randn(S, hq, dh), randn(S, hkv, dh), randn(S, hkv, dh), randn(S, hq, dh)
+    # (1) without the rowsum term the key gradients no longer sum to zero
+    orig_exp = np.exp
+
+    def bwd_no_d(q, k, v, do, causal=True):
+        sc = 1.0 / math.sqrt(dh)
+        mask = ref.explicit_mask(np.arange(S), np.arange(S), causal)
+        dk = np.zeros_like(k)
+        for h in range(hq):
+            s = np.where(mask, (q[:, h] @ k[:, 0].T) * sc, -np.inf)
+            p = orig_exp(s - s.max(axis=1, keepdims=True))
+            p /= p.sum(axis=1, keepdims=True)
+            ds = p * (do[:, h] @ v[:, 0].T)          # planted: D dropped
+            dk[:, 0] += sc * ds.T @ q[:, h]
+        return dk
+
+    assert np.abs(bwd_no_d(q, k, v, do).sum(axis=0)).max() > 1e-6
+    assert np.abs(ref.attention_bwd(q, k, v, do)[1].sum(axis=0)).max() < 1e-10
+    # (2) a ring backward whose P uses a wrong normaliser (LSE off by ln 2)
+    # no longer equals the unsplit gradient
+    o_all, lse_all = ref.ring_attention(q, k, v, S, 2, "contiguous")
+    monkeypatch.setattr(ref, "ring_attention",
+                        lambda *a, **kw: (o_all, lse_all - np.log(2.0)))  # planted: wrong normaliser
+    bad = ref.ring_attention_bwd(q, k, v, do, S, 2, "contiguous")
+    monkeypatch.undo()
+    good = ref.attention_bwd(q, k, v, do)
+    assert not np.allclose(bad[0], good[0], atol=1e-6)

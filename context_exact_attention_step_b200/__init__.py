@@ -14,6 +14,8 @@ from .api import (  # noqa: F401
     set_profile_events,
     striped_reorder,
     lse_merge,
+    ring_attn_bwd,
+    ring_attn_bwd_workspace_size,
     ring_attn_fwd,
     ring_attn_workspace_size,
     ring_schedule,

@@ -289,6 +289,46 @@ def usp_attn_fwd(q, k, v, Pr, Pu, layout="contiguous", causal=True, cu_seqlens=N
     return o, lse
 
 
+def ring_attn_bwd_workspace_size(S, hq, hkv, dh, P, layout="contiguous", causal=True, cu_seqlens=None) -> int:
+    cu_p, n_docs, _keep = _cu_host(cu_seqlens)
+    out = ctypes.c_size_t(0)
+    check(lib().cp_ring_attn_bwd_workspace_size(S, hq, hkv, dh, P, _LAYOUTS[layout],
+                                                _lib.CP_MASK_CAUSAL if causal else _lib.CP_MASK_NONE, cu_p, n_docs,
+                                                ctypes.byref(out)))
+    return int(out.value)
+
+
+def ring_attn_bwd(q, k, v, o, lse, do, P, layout="contiguous", causal=True, cu_seqlens=None, cu_seqlens_dev=None,
+                  softmax_scale=0.0, dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """Gradients of ring_attn_fwd.  q [S, hq, dh], k, v [S, hkv, dh], do
+    [S, hq, dh] bf16 and the forward's o [S, hq, dh], lse [hq, S] fp32, all
+    CUDA and in the rank-major order of ``layout``.  Returns (dQ [S, hq, dh],
+    dK [S, hkv, dh], dV [S, hkv, dh]) fp32 in the same order."""
+    for n, t in (("q", q), ("k", k), ("v", v), ("do", do)):
+        _need_cuda(n, t, torch.bfloat16)
+    _need_cuda("o", o, torch.float32)
+    _need_cuda("lse", lse, torch.float32)
+    S, hq, dh = q.shape
+    hkv = k.shape[1]
+    cu_p, n_docs, cu_np = _cu_host(cu_seqlens)
+    if n_docs > 0 and cu_seqlens_dev is None:
+        cu_seqlens_dev = torch.from_numpy(cu_np).to(q.device)
+    if dq is None:
+        dq = torch.empty((S, hq, dh), device=q.device, dtype=torch.float32)
+    if dk is None:
+        dk = torch.empty((S, hkv, dh), device=q.device, dtype=torch.float32)
+    if dv is None:
+        dv = torch.empty((S, hkv, dh), device=q.device, dtype=torch.float32)
+    if workspace is None:
+        need = ring_attn_bwd_workspace_size(S, hq, hkv, dh, P, layout, causal, cu_seqlens)
+        workspace = torch.empty(max(need, 256), device=q.device, dtype=torch.uint8)
+    check(lib().cp_ring_attn_bwd(_vp(q), _vp(k), _vp(v), _vp(o), _vp(lse), _vp(do), S, hq, hkv, dh, P,
+                                 _LAYOUTS[layout], _lib.CP_MASK_CAUSAL if causal else _lib.CP_MASK_NONE, cu_p,
+                                 _vp(cu_seqlens_dev), n_docs, float(softmax_scale), _vp(dq), _vp(dk), _vp(dv),
+                                 _vp(workspace), workspace.numel(), _stream(stream)))
+    return dq, dk, dv
+
+
 def ring_schedule(S, P, layout="contiguous", causal=True, cu_seqlens=None):
     """Host-only view of the ring-step schedule: arrays of P*P entries indexed
     r*P + t (see cp_ring_schedule)."""

@@ -21,7 +21,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libcp_attn.so")
 
-SOURCES = ["attn_fwd.cu", "merge.cu", "permute.cu", "api.cu", "scheduler.cpp", "runtime.cpp", "ring_noalloc.cu", "selftest.cu"]
+SOURCES = ["attn_fwd.cu", "attn_bwd.cu", "merge.cu", "permute.cu", "api.cu", "scheduler.cpp", "runtime.cpp", "ring_noalloc.cu", "selftest.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-I" + INCLUDE, "-I" + CSRC]
 

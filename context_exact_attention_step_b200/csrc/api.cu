@@ -31,6 +31,10 @@ cudaError_t launch_zigzag(const void* in, void* out, int P, int batch, size_t ch
 cudaError_t launch_f32_to_bf16(const float* in, void* out, size_t n, cudaStream_t st);
 cudaError_t launch_striped(const void* in, void* out, int P, int S, int batch, size_t row_bytes, int inverse,
                            cudaStream_t st);
+cudaError_t launch_bwd_prep(int dh, const float* o, const void* dout, const float* lse, int S, int hq, float* lg,
+                            float* dd, cudaStream_t st);
+cudaError_t launch_bwd(int dh, const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
+                       const CUtensorMap& tv, const cp_bwd_plan& plan, bool dq_side, cudaStream_t st);
 std::atomic<uint64_t>& launch_counter();
 }  // namespace cp
 
@@ -693,6 +697,143 @@ cp_status cp_usp_attn_fwd(const void* q, const void* k, const void* v, int S, in
   }
   if ((s = run_merge(tasks, hg, dh, o, lse, S, nullptr, st, hq)) != CP_OK) return s;
   record(g_ev_merge_end, st);
+  return ok();
+}
+
+// ------------------------------------------------------------------ backward
+static size_t bwd_workspace(int S, int hq) { return 2 * align256((size_t)S * hq * sizeof(float)); }
+
+cp_status cp_ring_attn_bwd_workspace_size(int S, int hq, int hkv, int dh, int P, cp_layout layout, cp_mask mask,
+                                          const int32_t* cu_seqlens_host, int n_docs, size_t* bytes) {
+  cp_status s;
+  if (!bytes) return fail(CP_ERR_INVALID_ARG, "bytes is NULL");
+  if ((s = ring_check(S, hq, hkv, dh, P, layout, mask, CP_BF16, cu_seqlens_host, n_docs)) != CP_OK) return s;
+  *bytes = bwd_workspace(S, hq);
+  return ok();
+}
+
+namespace {
+struct BwdItem {
+  uint32_t code;
+  int64_t cost;
+};
+
+// Own 128-row tiles of every rank (dq_side) or shard, ordered by the number
+// of (q, k) pairs they admit, heaviest first.
+std::vector<uint32_t> bwd_items(const cp_bwd_plan& pl, bool dq_side, const Docs& docs) {
+  std::vector<BwdItem> v;
+  for (int a = 0; a < pl.P; ++a)
+    for (int sg = 0; sg < pl.nseg[a]; ++sg) {
+      const cp_seg& own = pl.seg[a][sg];
+      for (int t = 0; t * 128 < own.len; ++t) {
+        const int pos = own.pos + t * 128, len = std::min(128, own.len - t * 128);
+        int64_t cost = 0;
+        for (int b = 0; b < pl.P; ++b)
+          for (int x = 0; x < pl.nseg[b]; ++x) {
+            const cp_seg& other = pl.seg[b][x];
+            // striped: a key of shard j sits one position later for rank r < j
+            if (dq_side) {
+              const int shift = (pl.striped && b > a) ? 1 : 0;
+              cost += count_admitted(pos, len, other.pos + shift, other.len, pl.causal != 0, docs);
+            } else {
+              const int shift = (pl.striped && a > b) ? 1 : 0;
+              cost += count_admitted(other.pos, other.len, pos + shift, len, pl.causal != 0, docs);
+            }
+          }
+        v.push_back({((uint32_t)a << 24) | ((uint32_t)sg << 23) | (uint32_t)t, cost});
+      }
+    }
+  std::stable_sort(v.begin(), v.end(), [](const BwdItem& x, const BwdItem& y) { return x.cost > y.cost; });
+  std::vector<uint32_t> out;
+  out.reserve(v.size());
+  for (const BwdItem& x : v) out.push_back(x.code);
+  return out;
+}
+}  // namespace
+
+cp_status cp_ring_attn_bwd(const void* q, const void* k, const void* v, const float* o, const float* lse,
+                           const void* dout, int S, int hq, int hkv, int dh, int P, cp_layout layout, cp_mask mask,
+                           const int32_t* cu_seqlens_host, const int32_t* cu_seqlens_dev, int n_docs,
+                           float softmax_scale, float* dq, float* dk, float* dv, void* workspace, size_t ws_bytes,
+                           void* stream) {
+  cp_status s;
+  if ((s = ring_check(S, hq, hkv, dh, P, layout, mask, CP_BF16, cu_seqlens_host, n_docs)) != CP_OK) return s;
+  CP_CHECK_PTR(q);
+  CP_CHECK_PTR(k);
+  CP_CHECK_PTR(v);
+  CP_CHECK_PTR(o);
+  CP_CHECK_PTR(lse);
+  CP_CHECK_PTR(dout);
+  CP_CHECK_PTR(dq);
+  CP_CHECK_PTR(dk);
+  CP_CHECK_PTR(dv);
+  if (P > CP_BWD_MAX_RANKS) return fail(CP_ERR_UNSUPPORTED, "P = %d (backward supports 1..%d)", P, CP_BWD_MAX_RANKS);
+  if (n_docs > 0 && !cu_seqlens_dev) return fail(CP_ERR_INVALID_ARG, "n_docs > 0 needs cu_seqlens_dev");
+  const size_t need = bwd_workspace(S, hq);
+  if (!workspace || ws_bytes < need)
+    return fail(CP_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws_bytes);
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return fail(CP_ERR_ALIGNMENT, "workspace is not 256-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* lg = static_cast<float*>(workspace);
+  float* dd = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + align256((size_t)S * hq * sizeof(float)));
+
+  CUtensorMap tq, tdo, tk, tv;
+  if ((s = make_map(&tq, q, S, (int64_t)hq * dh, 128)) != CP_OK) return s;
+  if ((s = make_map(&tdo, dout, S, (int64_t)hq * dh, 128)) != CP_OK) return s;
+  if ((s = make_map(&tk, k, S, (int64_t)hkv * dh, 128)) != CP_OK) return s;
+  if ((s = make_map(&tv, v, S, (int64_t)hkv * dh, 128)) != CP_OK) return s;
+  uint32_t* err = nullptr;
+  if ((s = err_word(&err)) != CP_OK) return s;
+
+  static cp_bwd_plan plan;  // large POD: keep it off the stack
+  static std::mutex plan_mu;
+  std::lock_guard<std::mutex> lk(plan_mu);
+  memset(&plan, 0, sizeof(plan));
+  const Layout lay = layout == CP_LAYOUT_ZIGZAG ? Layout::Zigzag
+                     : layout == CP_LAYOUT_STRIPED ? Layout::Striped
+                                                   : Layout::Contiguous;
+  plan.P = P;
+  plan.hq = hq;
+  plan.hkv = hkv;
+  plan.causal = mask == CP_MASK_CAUSAL ? 1 : 0;
+  plan.striped = lay == Layout::Striped ? 1 : 0;
+  plan.n_docs = n_docs;
+  plan.cu_seqlens = cu_seqlens_dev;
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)dh);
+  plan.scale = scale;
+  plan.scale_log2 = scale * 1.4426950408889634f;
+  plan.S = S;
+  for (int r = 0; r < P; ++r) {
+    const std::vector<Seg> segs = shard_segments(S, P, lay, r);
+    plan.nseg[r] = (int)segs.size();
+    for (size_t x = 0; x < segs.size(); ++x) plan.seg[r][x] = {segs[x].buf_row, segs[x].pos, segs[x].len, 0};
+  }
+  plan.lg = lg;
+  plan.dd = dd;
+  plan.dq = dq;
+  plan.dk = dk;
+  plan.dv = dv;
+  plan.err = err;
+  Docs docs;
+  if (cu_seqlens_host && n_docs > 0) {
+    docs.cu = cu_seqlens_host;
+    docs.n = n_docs;
+  }
+  cudaError_t e = launch_bwd_prep(dh, o, dout, lse, S, hq, lg, dd, st);
+  if (e != cudaSuccess) return cuda_fail(e, "backward prep launch");
+  record(g_ev_attn_begin, st);
+  for (int side = 0; side < 2; ++side) {
+    const bool dq_side = side == 0;
+    const std::vector<uint32_t> items = bwd_items(plan, dq_side, docs);
+    for (size_t base = 0; base < items.size(); base += CP_BWD_MAX_ITEMS) {
+      const size_t cnt = std::min(items.size() - base, (size_t)CP_BWD_MAX_ITEMS);
+      plan.n_items = (int)cnt;
+      std::copy(items.begin() + base, items.begin() + base + cnt, plan.items);
+      e = launch_bwd(dh, tq, tdo, tk, tv, plan, dq_side, st);
+      if (e != cudaSuccess) return cuda_fail(e, dq_side ? "backward dQ launch" : "backward dK/dV launch");
+    }
+  }
+  record(g_ev_attn_end, st);
   return ok();
 }
 

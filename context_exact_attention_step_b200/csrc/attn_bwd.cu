@@ -1,0 +1,933 @@
+// Backward of the ring-step block attention (sm_100a).
+//
+// The pages define the forward only; the backward is the gradient of that
+// exact attention for an upstream dO.  Ring form: the forward's merged O and
+// LSE of every rank are kept, and at ring step t rank r, holding key/value
+// shard j = (r - t) mod P, contributes with
+//     P_rj  = exp(scale Q_r K_j^T - LSE_r)      (the merged LSE, so P_rj is
+//                                               the true slice of softmax)
+//     D_r   = rowsum(dO_r * O_r)
+//     dS_rj = P_rj * (dO_r V_j^T - D_r)
+//     dQ_r += scale dS_rj K_j,  dK_j += scale dS_rj^T Q_r,  dV_j += P_rj^T dO_r.
+// Differentiating the LSE merge ("序列並行（Sequence Parallelism）" concept
+// page (compassingai), 技術原理 §二, the block recurrence) together with each
+// pair's own normalisation gives exactly this, so the merge needs no backward
+// kernel of its own.  Masks follow each block's global positions as in the
+// forward ("Context Parallelism" write-up (pwwt.cn) §3.3).
+//
+// With the P ranks on one GPU the contributions are summed on chip instead
+// of travelling around the ring:
+//   * bwd_prep_kernel: D and LSE * log2(e) for every (row, head)   (HBM-bound)
+//   * attn_bwd_dq_kernel: one CTA per (128-row query tile of rank r, query
+//     head) walks the key/value tiles of shards (r - t) mod P, t = 0..P-1,
+//     and accumulates dQ in tensor memory;
+//   * attn_bwd_dkdv_kernel: one CTA per (128-row key/value tile of shard j,
+//     KV head) walks the query tiles of ranks (j + t) mod P and every query
+//     head of the group, and accumulates dK and dV in tensor memory.
+// No atomics: every output row is written once by one CTA.
+//
+// CTA layout of both tensor-core kernels (256 threads, one CTA per SM):
+//   warp 0      TMA producer
+//   warp 1      tcgen05.mma issuer (one elected lane) and TMEM owner
+//   warps 2-3   idle
+//   warps 4-7   element-wise stage, one own row per thread (TMEM lane)
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math_constants.h>
+
+#include <atomic>
+
+#include "plan.h"
+#include "sm100_ptx.cuh"
+
+namespace cp {
+
+std::atomic<uint64_t>& launch_counter();
+
+namespace {
+
+constexpr int kBwdThreads = 256;
+constexpr int kNoLo = -(1 << 30);
+constexpr int kNoHi = (1 << 30);
+constexpr float kLog2e = 1.4426950408889634f;
+// Every wait of these kernels is on the CTA's own pipeline and lasts
+// microseconds; half a second means the CTA is stuck, so it gives up.
+constexpr uint64_t kWaitNs = 500000000ull;
+
+__device__ __forceinline__ int bdoc_index(const int32_t* __restrict__ cu, int n_docs, int x) {
+  int lo = 0, hi = n_docs - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(cu + mid) <= x) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+__device__ __forceinline__ int bdoc_start(const int32_t* __restrict__ cu, int n_docs, int x) {
+  return __ldg(cu + bdoc_index(cu, n_docs, x));
+}
+__device__ __forceinline__ int bdoc_last(const int32_t* __restrict__ cu, int n_docs, int x) {
+  return __ldg(cu + bdoc_index(cu, n_docs, x) + 1) - 1;
+}
+
+template <int DH>
+struct BwdTile {
+  static constexpr int kBoxes = DH / 64;       // 128-byte column boxes per row
+  static constexpr int kBoxBytes = 128 * 128;  // 128 rows x 128 bytes
+  static constexpr int kTileBytes = kBoxes * kBoxBytes;
+};
+
+struct Own {
+  int rank, buf_row0, pos0, valid;
+};
+
+__device__ __forceinline__ void decode_own(const cp_bwd_plan& pl, uint32_t item, Own& o) {
+  o.rank = (int)(item >> 24);
+  const int sg = (int)((item >> 23) & 1u);
+  const int tile = (int)(item & 0x7FFFFFu);
+  const cp_seg& s = pl.seg[o.rank][sg];
+  o.buf_row0 = s.buf_row + tile * 128;
+  o.pos0 = s.pos + tile * 128;
+  o.valid = min(128, s.len - tile * 128);
+}
+
+// ------------------------------------------------------------------ dQ side
+struct KvTile {
+  int buf_row, pos, valid;
+  bool full;
+};
+
+// Key/value tiles seen by one query tile of rank r, in ring-step order.
+// Every role of the CTA runs its own copy and sees the same sequence.
+struct DqIter {
+  const cp_bwd_plan* pl;
+  int r, t, sg, tl;
+  int vis_lo, vis_hi, full_lo, full_hi;
+
+  __device__ void init(const cp_bwd_plan& p, const Own& own) {
+    pl = &p;
+    r = own.rank;
+    t = sg = tl = 0;
+    const int qa = own.pos0, qb = own.pos0 + own.valid - 1;
+    const bool docs = p.n_docs > 0;
+    vis_lo = docs ? bdoc_start(p.cu_seqlens, p.n_docs, qa) : kNoLo;
+    full_lo = docs ? bdoc_start(p.cu_seqlens, p.n_docs, qb) : kNoLo;
+    vis_hi = p.causal ? qb : (docs ? bdoc_last(p.cu_seqlens, p.n_docs, qb) : kNoHi);
+    full_hi = p.causal ? qa : (docs ? bdoc_last(p.cu_seqlens, p.n_docs, qa) : kNoHi);
+  }
+
+  __device__ bool next(KvTile& out) {
+    const int P = pl->P;
+    while (t < P) {
+      const int j = ((r - t) % P + P) % P;
+      if (sg >= pl->nseg[j]) {
+        ++t;
+        sg = tl = 0;
+        continue;
+      }
+      const cp_seg& s = pl->seg[j][sg];
+      const int off = tl * 128;
+      if (off >= s.len) {
+        ++sg;
+        tl = 0;
+        continue;
+      }
+      const int ka = s.pos + ((pl->striped && j > r) ? 1 : 0) + off;
+      if (ka > vis_hi) {  // positions grow along a segment
+        ++sg;
+        tl = 0;
+        continue;
+      }
+      ++tl;
+      const int valid = min(128, s.len - off);
+      const int kb = ka + valid - 1;
+      if (kb >= vis_lo && ka <= vis_hi) {
+        out.buf_row = s.buf_row + off;
+        out.pos = ka;
+        out.valid = valid;
+        out.full = valid == 128 && ka >= full_lo && kb <= full_hi;
+        return true;
+      }
+    }
+    return false;
+  }
+};
+
+template <int DH>
+struct DqCfg {
+  using T = BwdTile<DH>;
+  static constexpr int kStages = DH == 128 ? 4 : 8;
+  static constexpr int kSmemBytes = 1024 + 2 * T::kTileBytes + kStages * T::kTileBytes + 256;
+  // TMEM: S | dP (two buffers; dS is written over its dP) | dQ
+  static constexpr uint32_t kColS = 0, kColD0 = 128, kColD1 = 256, kColQ = 384;
+};
+
+template <int DH>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                       const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                       const __grid_constant__ cp_bwd_plan plan) {
+  using C = DqCfg<DH>;
+  using T = BwdTile<DH>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sDO = smem + T::kTileBytes;
+  uint8_t* sKV = smem + 2 * T::kTileBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + C::kStages * T::kTileBytes);
+  const int B_QD = 0, B_FULL = 1, B_EMPTY = 1 + C::kStages, B_S = 1 + 2 * C::kStages, B_DP = B_S + 1,
+            B_SC = B_DP + 1, B_DS = B_SC + 1, B_ACC = B_DS + 1, B_DRAIN = B_ACC + 1, B_COUNT = B_DRAIN + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + B_COUNT);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  auto bar = [&](int i) { return smem_addr(bars + i); };
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  uint32_t* err = plan.err;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(B_QD), 1);
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(bar(B_FULL + s), 1);
+      mbar_init(bar(B_EMPTY + s), 1);
+    }
+    mbar_init(bar(B_S), 1);
+    mbar_init(bar(B_DP), 1);
+    mbar_init(bar(B_SC), 4);  // one arrive per element-wise warp
+    mbar_init(bar(B_DS), 4);
+    mbar_init(bar(B_ACC), 1);
+    mbar_init(bar(B_DRAIN), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_do);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(tmem_holder), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  const int h = blockIdx.x % plan.hq;
+  const int hk = h / (plan.hq / plan.hkv);
+  Own own;
+  decode_own(plan, plan.items[blockIdx.x / plan.hq], own);
+  auto col_d = [](int j) { return (j & 1) ? C::kColD1 : C::kColD0; };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    mbar_arrive_expect_tx_elect(bar(B_QD), 2 * T::kTileBytes);
+    for (int b = 0; b < T::kBoxes; ++b) {
+      tma_load_2d_elect(smem_addr(sQ + b * T::kBoxBytes), &tm_q, h * DH + b * 64, own.buf_row0, bar(B_QD));
+      tma_load_2d_elect(smem_addr(sDO + b * T::kBoxBytes), &tm_do, h * DH + b * 64, own.buf_row0, bar(B_QD));
+    }
+    DqIter it;
+    it.init(plan, own);
+    KvTile kt;
+    uint32_t c = 0;
+    bool ok = true;
+    while (ok && it.next(kt)) {
+      for (int w = 0; w < 2 && ok; ++w) {
+        const int slot = c % C::kStages;
+        const uint32_t ph = (c / C::kStages) & 1u;
+        ok = mbar_wait_warp(bar(B_EMPTY + slot), ph ^ 1u, abort_flag, err, kWaitNs);
+        if (!ok) break;
+        mbar_arrive_expect_tx_elect(bar(B_FULL + slot), T::kTileBytes);
+        const CUtensorMap* m = w == 0 ? &tm_k : &tm_v;
+        for (int b = 0; b < T::kBoxes; ++b)
+          tma_load_2d_elect(smem_addr(sKV + slot * T::kTileBytes + b * T::kBoxBytes), m, hk * DH + b * 64,
+                            kt.buf_row, bar(B_FULL + slot));
+        ++c;
+      }
+    }
+    const uint32_t first = c > (uint32_t)C::kStages ? c - C::kStages : 0u;
+    for (uint32_t i = first; i < c; ++i)
+      mbar_wait_warp(bar(B_FULL + i % C::kStages), (i / C::kStages) & 1u, abort_flag, nullptr, 1000000000ull);
+    mbar_wait_warp(bar(B_QD), 0, abort_flag, nullptr, 1000000000ull);
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    constexpr uint32_t idesc_ss = idesc_bf16_f32(128, 128, false);
+    constexpr uint32_t idesc_dq = idesc_bf16_f32(128, DH, true);
+    const uint32_t sq = smem_addr(sQ), sdo = smem_addr(sDO), skv = smem_addr(sKV);
+    // D[col] = A B^T over dh, both operands K-major 128-row tiles
+    auto issue_ss = [&](uint32_t dcol, uint32_t a_base, uint32_t b_base) {
+#pragma unroll
+      for (int kk = 0; kk < DH / 16; ++kk) {
+        const uint32_t box = kk >> 2, koff = (kk & 3) * 32;
+        const uint64_t a = sdesc_sw128(a_base + box * T::kBoxBytes + koff, 16, 1024);
+        const uint64_t b = sdesc_sw128(b_base + box * T::kBoxBytes + koff, 16, 1024);
+        tc_mma_ss_elect(tmem + dcol, a, b, idesc_ss, kk > 0 ? 1u : 0u);
+      }
+    };
+    // dQ += dS K: A = dS (bf16 in TMEM, 128 keys), B = the K tile read MN-major
+    auto issue_dq = [&](uint32_t acol, uint32_t kbase, bool acc) {
+#pragma unroll
+      for (int kk = 0; kk < 128 / 16; ++kk) {
+        const uint64_t b = sdesc_sw128(kbase + kk * 2048, T::kBoxBytes, 1024);
+        tc_mma_ts_elect(tmem + C::kColQ, tmem + acol + kk * 8, b, idesc_dq, (acc || kk > 0) ? 1u : 0u);
+      }
+    };
+    auto kslot = [&](int j) { return (2 * j) % C::kStages; };
+    auto kph = [&](int j) { return (uint32_t)(((2 * j) / C::kStages) & 1); };
+    auto vslot = [&](int j) { return (2 * j + 1) % C::kStages; };
+    auto vph = [&](int j) { return (uint32_t)(((2 * j + 1) / C::kStages) & 1); };
+    auto slot_addr = [&](int s) { return skv + (uint32_t)s * T::kTileBytes; };
+
+    bool ok = mbar_wait_warp(bar(B_QD), 0, abort_flag, err, kWaitNs);
+    DqIter it;
+    it.init(plan, own);
+    KvTile cur, nxt;
+    bool have = ok && it.next(cur);
+    if (have) {
+      ok = mbar_wait_warp(bar(B_FULL + kslot(0)), kph(0), abort_flag, err, kWaitNs);
+      if (ok) {
+        tc_fence_after();
+        issue_ss(C::kColS, sq, slot_addr(kslot(0)));
+        tc_commit_elect(bar(B_S));
+        ok = mbar_wait_warp(bar(B_FULL + vslot(0)), vph(0), abort_flag, err, kWaitNs);
+      }
+      if (ok) {
+        tc_fence_after();
+        issue_ss(col_d(0), sdo, slot_addr(vslot(0)));
+        tc_commit_elect(bar(B_DP));
+        tc_commit_elect(bar(B_EMPTY + vslot(0)));
+      }
+      have = ok;
+    }
+    int j = 0;
+    while (have) {
+      const bool hn = it.next(nxt);
+      // S(j) has been read: S(j+1) may overwrite it
+      if (!(ok = mbar_wait_warp(bar(B_SC), j & 1u, abort_flag, err, kWaitNs))) break;
+      if (hn) {
+        if (!(ok = mbar_wait_warp(bar(B_FULL + kslot(j + 1)), kph(j + 1), abort_flag, err, kWaitNs))) break;
+        tc_fence_after();
+        issue_ss(C::kColS, sq, slot_addr(kslot(j + 1)));
+        tc_commit_elect(bar(B_S));
+      }
+      if (!(ok = mbar_wait_warp(bar(B_DS), j & 1u, abort_flag, err, kWaitNs))) break;
+      tc_fence_after();
+      issue_dq(col_d(j), slot_addr(kslot(j)), j > 0);
+      tc_commit_elect(bar(B_EMPTY + kslot(j)));
+      if (hn) {
+        if (!(ok = mbar_wait_warp(bar(B_FULL + vslot(j + 1)), vph(j + 1), abort_flag, err, kWaitNs))) break;
+        tc_fence_after();
+        issue_ss(col_d(j + 1), sdo, slot_addr(vslot(j + 1)));
+        tc_commit_elect(bar(B_DP));
+        tc_commit_elect(bar(B_EMPTY + vslot(j + 1)));
+      }
+      cur = nxt;
+      have = hn;
+      ++j;
+    }
+    tc_commit_elect(bar(B_ACC));
+    tc_commit_elect(bar(B_DRAIN));
+    mbar_wait_warp(bar(B_DRAIN), 0, abort_flag, nullptr, 1000000000ull);
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ element-wise
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const bool rvalid = row < own.valid;
+    const int qpos = own.pos0 + row;
+    const bool docs = plan.n_docs > 0;
+    const size_t vec = (size_t)h * plan.S + own.buf_row0 + row;
+    const float neg_lg = rvalid ? -__ldg(plan.lg + vec) : 0.f;
+    const float dd = rvalid ? __ldg(plan.dd + vec) : 0.f;
+    const int row_lo = rvalid ? (docs ? bdoc_start(plan.cu_seqlens, plan.n_docs, qpos) : kNoLo) : kNoHi;
+    const int row_hi =
+        rvalid ? (plan.causal ? qpos : (docs ? bdoc_last(plan.cu_seqlens, plan.n_docs, qpos) : kNoHi)) : kNoLo;
+    const uint64_t c2 = f2_pack(plan.scale_log2, plan.scale_log2);
+    const uint64_t nl2 = f2_pack(neg_lg, neg_lg);
+    const uint64_t nd2 = f2_pack(-dd, -dd);
+    DqIter it;
+    it.init(plan, own);
+    KvTile kt;
+    int j = 0;
+    bool ok = true;
+    while (it.next(kt)) {
+      ok = mbar_wait(bar(B_S), j & 1u, abort_flag, err, kWaitNs);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t s[128];
+      const uint32_t tS = tmem + lane_base + C::kColS;
+      tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+      tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+      tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
+      tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
+      tc_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_SC));
+      if (!kt.full) {
+        const int clo = row_lo - kt.pos;
+        const int chi = min(row_hi - kt.pos, kt.valid - 1);
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c < clo || c > chi) s[c] = __float_as_uint(-CUDART_INF_F);
+      }
+      // P = 2^(S * scale * log2(e) - LSE * log2(e)), in place
+#pragma unroll
+      for (int c = 0; c < 128; c += 2) {
+        float x0, x1;
+        f2_unpack(f2_fma(f2_pack(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), c2, nl2), x0, x1);
+        s[c] = __float_as_uint(ex2_approx(x0));
+        s[c + 1] = __float_as_uint(ex2_approx(x1));
+      }
+      ok = mbar_wait(bar(B_DP), j & 1u, abort_flag, err, kWaitNs);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t tD = tmem + lane_base + col_d(j);
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t d[32];
+        tmem_ld32(tD + ch * 32, d);
+        tc_wait_ld();
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int c = ch * 32 + 2 * i;
+          const uint64_t t = f2_add(f2_pack(__uint_as_float(d[2 * i]), __uint_as_float(d[2 * i + 1])), nd2);
+          float a, b;
+          f2_unpack(f2_mul(f2_pack(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), t), a, b);
+          w[i] = pack_bf16x2(a, b);
+        }
+        // columns [16 ch, 16 ch + 16) of this buffer have already been read
+        tmem_st16(tD + ch * 16, w);
+      }
+      tc_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_DS));
+      ++j;
+    }
+    if (ok) {
+      ok = mbar_wait(bar(B_ACC), 0, abort_flag, err, kWaitNs);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    if (ok) {
+      tc_fence_after();
+      float* dst = plan.dq + ((size_t)(own.buf_row0 + row) * plan.hq + h) * DH;
+#pragma unroll 1
+      for (int ch = 0; ch < DH / 32; ++ch) {
+        uint32_t o[32];
+        if (j > 0) {
+          tmem_ld32(tmem + lane_base + C::kColQ + ch * 32, o);
+          tc_wait_ld();
+        }
+        if (rvalid) {
+          float4* d4 = reinterpret_cast<float4*>(dst + ch * 32);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            float4 v;
+            v.x = j > 0 ? __uint_as_float(o[4 * i + 0]) * plan.scale : 0.f;
+            v.y = j > 0 ? __uint_as_float(o[4 * i + 1]) * plan.scale : 0.f;
+            v.z = j > 0 ? __uint_as_float(o[4 * i + 2]) * plan.scale : 0.f;
+            v.w = j > 0 ? __uint_as_float(o[4 * i + 3]) * plan.scale : 0.f;
+            d4[i] = v;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------ dK/dV side
+struct QTile {
+  int buf_row, pos, valid, h, r;
+  bool full;
+};
+
+// Query tiles seen by one key/value tile of shard j: every query head of the
+// KV head's group, then the ranks (j + t) mod P that hold shard j at ring
+// step t, then their tiles.
+struct KvIter {
+  const cp_bwd_plan* pl;
+  int j, hk, g, t, sg, tl;
+  int ka0, kb0;                    // own positions without the striped shift
+  int lo0, hi0, flo0, fhi0;        // windows of admitted query positions
+
+  __device__ void init(const cp_bwd_plan& p, const Own& own, int kv_head) {
+    pl = &p;
+    j = own.rank;
+    hk = kv_head;
+    g = t = sg = tl = 0;
+    ka0 = own.pos0;
+    kb0 = own.pos0 + own.valid - 1;
+    const bool docs = p.n_docs > 0;
+    // a key k admits queries q >= k (causal) inside its document
+    lo0 = p.causal ? ka0 : (docs ? bdoc_start(p.cu_seqlens, p.n_docs, ka0) : kNoLo);
+    hi0 = docs ? bdoc_last(p.cu_seqlens, p.n_docs, kb0) : kNoHi;
+    flo0 = p.causal ? kb0 : (docs ? bdoc_start(p.cu_seqlens, p.n_docs, kb0) : kNoLo);
+    fhi0 = docs ? bdoc_last(p.cu_seqlens, p.n_docs, ka0) : kNoHi;
+  }
+
+  __device__ bool next(QTile& out) {
+    const int P = pl->P;
+    const int group = pl->hq / pl->hkv;
+    while (g < group) {
+      if (t >= P) {
+        ++g;
+        t = sg = tl = 0;
+        continue;
+      }
+      const int r = (j + t) % P;
+      if (sg >= pl->nseg[r]) {
+        ++t;
+        sg = tl = 0;
+        continue;
+      }
+      const cp_seg& s = pl->seg[r][sg];
+      const int off = tl * 128;
+      if (off >= s.len) {
+        ++sg;
+        tl = 0;
+        continue;
+      }
+      const int shift = (pl->striped && pl->causal && j > r) ? 1 : 0;
+      const int qa = s.pos + off;
+      if (qa > hi0) {  // positions grow along a segment
+        ++sg;
+        tl = 0;
+        continue;
+      }
+      ++tl;
+      const int valid = min(128, s.len - off);
+      const int qb = qa + valid - 1;
+      if (qb >= lo0 + shift && qa <= hi0) {
+        out.buf_row = s.buf_row + off;
+        out.pos = qa;
+        out.valid = valid;
+        out.h = hk * group + g;
+        out.r = r;
+        out.full = valid == 128 && qa >= flo0 + shift && qb <= fhi0;
+        return true;
+      }
+    }
+    return false;
+  }
+};
+
+template <int DH>
+struct DkvCfg {
+  using T = BwdTile<DH>;
+  static constexpr int kStages = DH == 128 ? 2 : 4;
+  static constexpr int kStageBytes = 2 * T::kTileBytes;  // Q and dO tiles
+  static constexpr int kVecBytes = 2 * 128 * 4;          // -LSE*log2(e) and D of the 128 query rows
+  static constexpr int kSmemBytes =
+      1024 + 2 * T::kTileBytes + kStages * kStageBytes + kStages * kVecBytes + 256;
+  // TMEM: two 128-column buffers (S^T with P^T and dS^T written over it, and
+  // dP^T, alternating per query tile) | dV | dK
+  static constexpr uint32_t kColDV = 256, kColDK = 256 + DH;
+};
+
+template <int DH>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                         const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                         const __grid_constant__ cp_bwd_plan plan) {
+  using C = DkvCfg<DH>;
+  using T = BwdTile<DH>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sK = smem;
+  uint8_t* sV = smem + T::kTileBytes;
+  uint8_t* sStage = smem + 2 * T::kTileBytes;
+  float* sVec = reinterpret_cast<float*>(sStage + C::kStages * C::kStageBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sVec) + C::kStages * C::kVecBytes);
+  const int B_KV = 0, B_FULL = 1, B_EMPTY = 1 + C::kStages, B_S = 1 + 2 * C::kStages, B_DP = B_S + 1,
+            B_P = B_DP + 1, B_DS = B_P + 1, B_ACC = B_DS + 1, B_DRAIN = B_ACC + 1, B_COUNT = B_DRAIN + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + B_COUNT);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  auto bar = [&](int i) { return smem_addr(bars + i); };
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  uint32_t* err = plan.err;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(B_KV), 1);
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(bar(B_FULL + s), 1 + 32);  // the copy's expect_tx plus one arrive per producer lane
+      mbar_init(bar(B_EMPTY + s), 1);
+    }
+    mbar_init(bar(B_S), 1);
+    mbar_init(bar(B_DP), 1);
+    mbar_init(bar(B_P), 4);
+    mbar_init(bar(B_DS), 4);
+    mbar_init(bar(B_ACC), 1);
+    mbar_init(bar(B_DRAIN), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_do);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(tmem_holder), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  const int hk = blockIdx.x % plan.hkv;
+  Own own;
+  decode_own(plan, plan.items[blockIdx.x / plan.hkv], own);
+  auto col_r = [](int i) { return (i & 1) ? 128u : 0u; };
+  auto stage_q = [&](int s) { return sStage + s * C::kStageBytes; };
+  auto stage_do = [&](int s) { return sStage + s * C::kStageBytes + T::kTileBytes; };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    mbar_arrive_expect_tx_elect(bar(B_KV), 2 * T::kTileBytes);
+    for (int b = 0; b < T::kBoxes; ++b) {
+      tma_load_2d_elect(smem_addr(sK + b * T::kBoxBytes), &tm_k, hk * DH + b * 64, own.buf_row0, bar(B_KV));
+      tma_load_2d_elect(smem_addr(sV + b * T::kBoxBytes), &tm_v, hk * DH + b * 64, own.buf_row0, bar(B_KV));
+    }
+    KvIter it;
+    it.init(plan, own, hk);
+    QTile qt;
+    uint32_t c = 0;
+    bool ok = true;
+    while (ok && it.next(qt)) {
+      const int slot = c % C::kStages;
+      const uint32_t ph = (c / C::kStages) & 1u;
+      ok = mbar_wait_warp(bar(B_EMPTY + slot), ph ^ 1u, abort_flag, err, kWaitNs);
+      if (!ok) break;
+      mbar_arrive_expect_tx_elect(bar(B_FULL + slot), 2 * T::kTileBytes);
+      for (int b = 0; b < T::kBoxes; ++b) {
+        tma_load_2d_elect(smem_addr(stage_q(slot) + b * T::kBoxBytes), &tm_q, qt.h * DH + b * 64, qt.buf_row,
+                          bar(B_FULL + slot));
+        tma_load_2d_elect(smem_addr(stage_do(slot) + b * T::kBoxBytes), &tm_do, qt.h * DH + b * 64, qt.buf_row,
+                          bar(B_FULL + slot));
+      }
+      // -LSE*log2(e) and D of the tile's query rows (0 past the tile's end)
+      float* vl = sVec + slot * (C::kVecBytes / 4);
+      float* vd = vl + 128;
+      const size_t base = (size_t)qt.h * plan.S + qt.buf_row;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int cidx = lane + 32 * i;
+        const bool in = cidx < qt.valid;
+        vl[cidx] = in ? -__ldg(plan.lg + base + cidx) : 0.f;
+        vd[cidx] = in ? __ldg(plan.dd + base + cidx) : 0.f;
+      }
+      mbar_arrive(bar(B_FULL + slot));  // release: the stores above are visible to the waiters
+      ++c;
+    }
+    const uint32_t first = c > (uint32_t)C::kStages ? c - C::kStages : 0u;
+    for (uint32_t i = first; i < c; ++i)
+      mbar_wait_warp(bar(B_FULL + i % C::kStages), (i / C::kStages) & 1u, abort_flag, nullptr, 1000000000ull);
+    mbar_wait_warp(bar(B_KV), 0, abort_flag, nullptr, 1000000000ull);
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    constexpr uint32_t idesc_ss = idesc_bf16_f32(128, 128, false);
+    constexpr uint32_t idesc_acc = idesc_bf16_f32(128, DH, true);
+    const uint32_t sk = smem_addr(sK), sv = smem_addr(sV);
+    auto issue_ss = [&](uint32_t dcol, uint32_t a_base, uint32_t b_base) {
+#pragma unroll
+      for (int kk = 0; kk < DH / 16; ++kk) {
+        const uint32_t box = kk >> 2, koff = (kk & 3) * 32;
+        const uint64_t a = sdesc_sw128(a_base + box * T::kBoxBytes + koff, 16, 1024);
+        const uint64_t b = sdesc_sw128(b_base + box * T::kBoxBytes + koff, 16, 1024);
+        tc_mma_ss_elect(tmem + dcol, a, b, idesc_ss, kk > 0 ? 1u : 0u);
+      }
+    };
+    // D[dcol] += A (bf16 in TMEM at acol, 128 query rows) x B (a 128-row
+    // query-side tile read MN-major)
+    auto issue_acc = [&](uint32_t dcol, uint32_t acol, uint32_t b_base, bool acc) {
+#pragma unroll
+      for (int kk = 0; kk < 128 / 16; ++kk) {
+        const uint64_t b = sdesc_sw128(b_base + kk * 2048, T::kBoxBytes, 1024);
+        tc_mma_ts_elect(tmem + dcol, tmem + acol + kk * 8, b, idesc_acc, (acc || kk > 0) ? 1u : 0u);
+      }
+    };
+    auto slot_of = [&](int i) { return i % C::kStages; };
+    auto ph_of = [&](int i) { return (uint32_t)((i / C::kStages) & 1); };
+
+    bool ok = mbar_wait_warp(bar(B_KV), 0, abort_flag, err, kWaitNs);
+    KvIter it;
+    it.init(plan, own, hk);
+    QTile cur, nxt;
+    bool have = ok && it.next(cur);
+    if (have) {
+      ok = mbar_wait_warp(bar(B_FULL + slot_of(0)), ph_of(0), abort_flag, err, kWaitNs);
+      if (ok) {
+        tc_fence_after();
+        issue_ss(col_r(0), sk, smem_addr(stage_q(slot_of(0))));
+        tc_commit_elect(bar(B_S));
+        issue_ss(col_r(1), sv, smem_addr(stage_do(slot_of(0))));
+        tc_commit_elect(bar(B_DP));
+      }
+      have = ok;
+    }
+    int i = 0;
+    while (have) {
+      const bool hn = it.next(nxt);
+      const int s = slot_of(i);
+      if (!(ok = mbar_wait_warp(bar(B_P), i & 1u, abort_flag, err, kWaitNs))) break;
+      tc_fence_after();
+      issue_acc(C::kColDV, col_r(i), smem_addr(stage_do(s)), i > 0);
+      if (!(ok = mbar_wait_warp(bar(B_DS), i & 1u, abort_flag, err, kWaitNs))) break;
+      tc_fence_after();
+      if (hn) {
+        if (!(ok = mbar_wait_warp(bar(B_FULL + slot_of(i + 1)), ph_of(i + 1), abort_flag, err, kWaitNs))) break;
+        tc_fence_after();
+        issue_ss(col_r(i + 1), sk, smem_addr(stage_q(slot_of(i + 1))));
+        tc_commit_elect(bar(B_S));
+      }
+      issue_acc(C::kColDK, col_r(i) + 64, smem_addr(stage_q(s)), i > 0);
+      tc_commit_elect(bar(B_EMPTY + s));
+      if (hn) {
+        // dP^T(i+1) goes where P^T(i) / dS^T(i) live: issued after the two
+        // MMAs that read them
+        issue_ss(col_r(i), sv, smem_addr(stage_do(slot_of(i + 1))));
+        tc_commit_elect(bar(B_DP));
+      }
+      cur = nxt;
+      have = hn;
+      ++i;
+    }
+    tc_commit_elect(bar(B_ACC));
+    tc_commit_elect(bar(B_DRAIN));
+    mbar_wait_warp(bar(B_DRAIN), 0, abort_flag, nullptr, 1000000000ull);
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ element-wise
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const bool rvalid = row < own.valid;
+    const int kpos = own.pos0 + row;
+    const bool docs = plan.n_docs > 0;
+    // admitted query positions of this key: [col_lo, col_hi]
+    const int lo0 = rvalid ? (plan.causal ? kpos : (docs ? bdoc_start(plan.cu_seqlens, plan.n_docs, kpos) : kNoLo))
+                           : kNoHi;
+    const int col_hi = rvalid ? (docs ? bdoc_last(plan.cu_seqlens, plan.n_docs, kpos) : kNoHi) : kNoLo;
+    const uint64_t c2 = f2_pack(plan.scale_log2, plan.scale_log2);
+    KvIter it;
+    it.init(plan, own, hk);
+    QTile qt;
+    int i = 0;
+    bool ok = true;
+    while (it.next(qt)) {
+      const int s = i % C::kStages;
+      const float* vl = sVec + s * (C::kVecBytes / 4);
+      const float* vd = vl + 128;
+      ok = mbar_wait(bar(B_S), i & 1u, abort_flag, err, kWaitNs);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      // P^T = 2^(S^T * scale * log2(e) - LSE_q * log2(e)), kept only as the
+      // bf16 pairs the dV MMA reads: S^T is read in two 64-column halves and
+      // P^T of half h is stored over columns [32 h, 32 h + 32), which hold S^T
+      // values already read.
+      const uint32_t tR = tmem + lane_base + col_r(i);
+      const int shift = (plan.striped && plan.causal && own.rank > qt.r && rvalid) ? 1 : 0;
+      const int clo = lo0 + shift - qt.pos;
+      const int chi = min(col_hi - qt.pos, qt.valid - 1);
+      uint32_t pk[64];
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        uint32_t sv[64];
+        tmem_ld32(tR + h2 * 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+        tmem_ld32(tR + h2 * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+        tc_wait_ld();
+        if (!qt.full) {
+#pragma unroll
+          for (int cc = 0; cc < 64; ++cc) {
+            const int c = h2 * 64 + cc;
+            if (c < clo || c > chi) sv[cc] = __float_as_uint(-CUDART_INF_F);
+          }
+        }
+#pragma unroll
+        for (int i2 = 0; i2 < 32; ++i2) {
+          const float2 l2 = *reinterpret_cast<const float2*>(vl + h2 * 64 + 2 * i2);
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[2 * i2]), __uint_as_float(sv[2 * i2 + 1])), c2,
+                           f2_pack(l2.x, l2.y)),
+                    x0, x1);
+          pk[h2 * 32 + i2] = pack_bf16x2(ex2_approx(x0), ex2_approx(x1));
+        }
+        tmem_st32(tR + h2 * 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[h2 * 32]));
+      }
+      tc_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_P));
+      ok = mbar_wait(bar(B_DP), i & 1u, abort_flag, err, kWaitNs);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      // dS^T = P^T * (dP^T - D_q) from the bf16 P^T, over columns [64, 128)
+      const uint32_t tD = tmem + lane_base + col_r(i + 1);
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t d[32];
+        tmem_ld32(tD + ch * 32, d);
+        tc_wait_ld();
+        uint32_t w[16];
+#pragma unroll
+        for (int i2 = 0; i2 < 16; ++i2) {
+          const int c = ch * 32 + 2 * i2;
+          const uint32_t pw = pk[ch * 16 + i2];
+          const float2 d2 = *reinterpret_cast<const float2*>(vd + c);
+          const uint64_t t = f2_add(f2_pack(__uint_as_float(d[2 * i2]), __uint_as_float(d[2 * i2 + 1])),
+                                    f2_pack(-d2.x, -d2.y));
+          float a, b;
+          f2_unpack(f2_mul(f2_pack(__uint_as_float(pw << 16), __uint_as_float(pw & 0xFFFF0000u)), t), a, b);
+          w[i2] = pack_bf16x2(a, b);
+        }
+        tmem_st16(tR + 64 + ch * 16, w);
+      }
+      tc_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_DS));
+      ++i;
+    }
+    if (ok) {
+      ok = mbar_wait(bar(B_ACC), 0, abort_flag, err, kWaitNs);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    if (ok) {
+      tc_fence_after();
+      const size_t orow = (size_t)(own.buf_row0 + row) * plan.hkv + hk;
+#pragma unroll 1
+      for (int which = 0; which < 2; ++which) {
+        float* dst = (which == 0 ? plan.dv : plan.dk) + orow * DH;
+        const uint32_t col = which == 0 ? C::kColDV : C::kColDK;
+        const float f = which == 0 ? 1.f : plan.scale;
+#pragma unroll 1
+        for (int ch = 0; ch < DH / 32; ++ch) {
+          uint32_t o[32];
+          if (i > 0) {
+            tmem_ld32(tmem + lane_base + col + ch * 32, o);
+            tc_wait_ld();
+          }
+          if (rvalid) {
+            float4* d4 = reinterpret_cast<float4*>(dst + ch * 32);
+#pragma unroll
+            for (int k4 = 0; k4 < 8; ++k4) {
+              float4 v;
+              v.x = i > 0 ? __uint_as_float(o[4 * k4 + 0]) * f : 0.f;
+              v.y = i > 0 ? __uint_as_float(o[4 * k4 + 1]) * f : 0.f;
+              v.z = i > 0 ? __uint_as_float(o[4 * k4 + 2]) * f : 0.f;
+              v.w = i > 0 ? __uint_as_float(o[4 * k4 + 3]) * f : 0.f;
+              d4[k4] = v;
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------ prep
+// D = rowsum(dO * O) and LSE * log2(e) per (row, head), one warp per pair.
+template <int DH>
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const float* __restrict__ o, const uint16_t* __restrict__ dout,
+                                                       const float* __restrict__ lse, int S, int hq,
+                                                       float* __restrict__ lg, float* __restrict__ dd) {
+  constexpr int E = DH / 32;
+  const long long item = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (item >= (long long)S * hq) return;
+  const int lane = threadIdx.x & 31;
+  const int row = (int)(item / hq);
+  const int h = (int)(item - (long long)row * hq);
+  const size_t base = ((size_t)row * hq + h) * DH + (size_t)lane * E;
+  float acc = 0.f;
+  if constexpr (E == 4) {
+    const float4 a = __ldcs(reinterpret_cast<const float4*>(o + base));
+    const uint2 b = __ldcs(reinterpret_cast<const uint2*>(dout + base));
+    acc = a.x * __uint_as_float(b.x << 16) + a.y * __uint_as_float(b.x & 0xFFFF0000u) +
+          a.z * __uint_as_float(b.y << 16) + a.w * __uint_as_float(b.y & 0xFFFF0000u);
+  } else {
+    const float2 a = __ldcs(reinterpret_cast<const float2*>(o + base));
+    const uint32_t b = __ldcs(reinterpret_cast<const unsigned int*>(dout + base));
+    acc = a.x * __uint_as_float(b << 16) + a.y * __uint_as_float(b & 0xFFFF0000u);
+  }
+#pragma unroll
+  for (int m = 16; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+  if (lane == 0) {
+    const size_t v = (size_t)h * S + row;
+    const float l = lse[v];
+    dd[v] = acc;
+    lg[v] = l == -CUDART_INF_F ? 0.f : l * kLog2e;
+  }
+}
+
+template <int DH>
+cudaError_t launch_bwd_dh(const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
+                          const CUtensorMap& tv, const cp_bwd_plan& plan, bool dq_side, cudaStream_t st) {
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(attn_bwd_dq_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         DqCfg<DH>::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(attn_bwd_dkdv_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             DkvCfg<DH>::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  if (plan.n_items <= 0) return cudaSuccess;
+  if (dq_side)
+    attn_bwd_dq_kernel<DH><<<plan.n_items * plan.hq, kBwdThreads, DqCfg<DH>::kSmemBytes, st>>>(tq, tdo, tk, tv, plan);
+  else
+    attn_bwd_dkdv_kernel<DH>
+        <<<plan.n_items * plan.hkv, kBwdThreads, DkvCfg<DH>::kSmemBytes, st>>>(tq, tdo, tk, tv, plan);
+  launch_counter()++;
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_prep(int dh, const float* o, const void* dout, const float* lse, int S, int hq, float* lg,
+                            float* dd, cudaStream_t st) {
+  const long long items = (long long)S * hq;
+  if (items <= 0) return cudaSuccess;
+  const unsigned grid = (unsigned)((items + 7) / 8);
+  if (dh == 128)
+    bwd_prep_kernel<128><<<grid, 256, 0, st>>>(o, static_cast<const uint16_t*>(dout), lse, S, hq, lg, dd);
+  else
+    bwd_prep_kernel<64><<<grid, 256, 0, st>>>(o, static_cast<const uint16_t*>(dout), lse, S, hq, lg, dd);
+  launch_counter()++;
+  return cudaGetLastError();
+}
+
+// dq_side: the dQ kernel (CTAs = items x hq); otherwise the dK/dV kernel
+// (CTAs = items x hkv).
+cudaError_t launch_bwd(int dh, const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
+                       const CUtensorMap& tv, const cp_bwd_plan& plan, bool dq_side, cudaStream_t st) {
+  if (dh == 128) return launch_bwd_dh<128>(tq, tdo, tk, tv, plan, dq_side, st);
+  return launch_bwd_dh<64>(tq, tdo, tk, tv, plan, dq_side, st);
+}
+
+}  // namespace cp

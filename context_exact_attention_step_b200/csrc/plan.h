@@ -81,3 +81,39 @@ struct cp_merge_plan {
   cp_merge_task tasks[CP_MAX_TASKS];
   cp_merge_input inputs[CP_MAX_INPUTS];
 };
+
+// ------------------------------------------------------------------ backward
+#define CP_BWD_MAX_RANKS 16
+#define CP_BWD_MAX_ITEMS 2048   // own 128-row tiles per backward launch
+
+// Backward of the ring over P ranks, run as two kernels: one CTA per
+// (own 128-row tile, head).  For the dQ kernel the own rows are a query tile
+// of rank r and the partners are the key/value shards j = (r - t) mod P of
+// the ring steps t = 0..P-1; for the dK/dV kernel the own rows are a key/value
+// tile of shard j and the partners are the ranks (j + t) mod P that hold it at
+// step t (and every query head of its group).
+//
+// item: (rank << 24) | (segment << 23) | tile, tile = 128-row tile index
+// inside the segment.  Striped layouts carry local row indices as positions;
+// a key of shard j seen from rank r then sits one position later when j > r.
+struct cp_bwd_plan {
+  int32_t P;
+  int32_t hq, hkv;
+  int32_t causal;
+  int32_t striped;
+  int32_t n_docs;
+  const int32_t* cu_seqlens;
+  float scale_log2;             // softmax_scale * log2(e)
+  float scale;
+  int32_t S;                    // rows of every buffer (row pitch of lg, dd)
+  int32_t nseg[CP_BWD_MAX_RANKS];
+  cp_seg seg[CP_BWD_MAX_RANKS][2];
+  const float* lg;              // [hq][S]: LSE * log2(e) (0 where LSE = -inf)
+  const float* dd;              // [hq][S]: rowsum(dO * O)
+  float* dq;                    // [S][hq][dh]
+  float* dk;                    // [S][hkv][dh]
+  float* dv;                    // [S][hkv][dh]
+  uint32_t* err;
+  int32_t n_items;
+  uint32_t items[CP_BWD_MAX_ITEMS];
+};

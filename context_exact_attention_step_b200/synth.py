@@ -9,6 +9,7 @@ Parallelism" write-up (pwwt.cn) §4.1):
   (seeds Q=1, K=2, V=3 unless overridden), multiplied by ``std`` (0.5 for the
   bf16 workloads, 1.0 for the tiny fp32 one), then rounded to bf16 with
   round-to-nearest-even when ``dtype`` is bf16.
+* Upstream gradient dO for the backward: same recipe as Q (seed 5).
 * Packed documents: integer lengths uniform on [lo, hi] inclusive drawn from
   seed 4 until their sum reaches the total; the last one is truncated so the
   lengths add up to exactly the total.  ``cu_seqlens`` are their int32 prefix
@@ -18,7 +19,7 @@ from __future__ import annotations
 
 import torch
 
-SEED_Q, SEED_K, SEED_V, SEED_DOCS = 1, 2, 3, 4
+SEED_Q, SEED_K, SEED_V, SEED_DOCS, SEED_DO = 1, 2, 3, 4, 5
 
 
 def normal(shape, seed, std=1.0, dtype=torch.bfloat16):

@@ -255,6 +255,41 @@ cp_status cp_usp_attn_fwd(const void* q, const void* k, const void* v, int S, in
                           void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * cp_ring_attn_bwd_workspace_size / cp_ring_attn_bwd -- gradients of the ring
+ * attention forward (cp_ring_attn_fwd) for an upstream gradient dO.  The pages
+ * define the forward; training also runs the backward (the DeepSpeed-Ulysses /
+ * ring-flash-attention how-to (2kiu.com), §4, checks memory after forward and
+ * backward), and this is the gradient of that exact attention in ring form:
+ * at step t rank r holds key/value shard j = (r - t) mod P and, with the
+ * forward's merged LSE_r and D_r = rowsum(dO_r * O_r),
+ *   P_rj = exp(scale Q_r K_j^T - LSE_r),  dS_rj = P_rj * (dO_r V_j^T - D_r),
+ *   dQ_r += scale dS_rj K_j,  dK_j += scale dS_rj^T Q_r,  dV_j += P_rj^T dO_r
+ * (masks by global position as in the forward; the LSE merge needs no
+ * separate backward because P_rj already uses the merged LSE).
+ *
+ * Inputs (device, in the rank-major order of `layout`, as given to and
+ * returned by cp_ring_attn_fwd): q [S][hq][dh], k, v [S][hkv][dh] bf16;
+ * o [S][hq][dh] fp32 and lse [hq][S] fp32 from the forward; dout [S][hq][dh]
+ * bf16.  Outputs (device, same order, fp32, fully overwritten): dq
+ * [S][hq][dh], dk and dv [S][hkv][dh].  GQA sums dk, dv over the query heads
+ * of each KV head.
+ *
+ * Runs a prep kernel (D and LSE*log2(e) into the workspace), a dQ kernel and
+ * a dK/dV kernel (tcgen05, accumulators in tensor memory, no atomics; the
+ * result does not depend on the launch order).  Workspace: caller-owned,
+ * 256-byte aligned, size from cp_ring_attn_bwd_workspace_size.
+ * Supported: bf16 only, everything else as cp_ring_attn_fwd.  Errors: as
+ * cp_ring_attn_fwd; nothing is launched on error.
+ */
+cp_status cp_ring_attn_bwd_workspace_size(int S, int hq, int hkv, int dh, int P, cp_layout layout, cp_mask mask,
+                                          const int32_t* cu_seqlens_host, int n_docs, size_t* bytes);
+cp_status cp_ring_attn_bwd(const void* q, const void* k, const void* v, const float* o, const float* lse,
+                           const void* dout, int S, int hq, int hkv, int dh, int P, cp_layout layout, cp_mask mask,
+                           const int32_t* cu_seqlens_host, const int32_t* cu_seqlens_dev, int n_docs,
+                           float softmax_scale, float* dq, float* dk, float* dv, void* workspace, size_t ws_bytes,
+                           void* stream);
+
+/*
  * Host-only inspection of the ring-step schedule (no GPU needed).  For every
  * rank r and step t (index r*P + t):
  *   src[r*P+t]        the key/value shard j = (r - t) mod P held at that step

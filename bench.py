@@ -43,6 +43,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "ring-attn fwd TFLOP/s & % BF16 tensor peak; a2a-permute GB/s % HBM"
+METRIC_BWD = "ring-attn bwd TFLOP/s (causal-effective, 2.5x the forward's FLOP) & % BF16 tensor peak"
 
 # DRAM traffic per launch of the block-attention kernel from an ncu capture,
 # keyed by the hash of the kernel source it was taken on (null once the
@@ -154,7 +155,7 @@ def max_over_ranks(x, ws):
 
 
 # ----------------------------------------------------------------- workloads
-def make_workload(name, seq_len=None):
+def make_workload(name, seq_len=None, pass_="fwd"):
     from context_exact_attention_step_b200 import api, synth
     cfg = dict(synth.CONFIGS[name])
     if seq_len:
@@ -217,9 +218,53 @@ def make_workload(name, seq_len=None):
         else:
             def step():
                 api.ring_attn_fwd(qd, kd, vd, P, layout, True, cu, cu_dev, o=o, lse=lse, workspace=ws)
+    if pass_ == "bwd":
+        make_bwd_step(w, api, synth, dev, ws)
+    else:
+        w["step"] = step
+        w["ws_bytes"] = ws.numel()
+    w["pass"] = pass_
+    return w
+
+
+def make_bwd_step(w, api, synth, dev, fwd_ws):
+    """Backward step of a ring workload: cp_ring_attn_bwd on inputs already in
+    the rank-major shard order, with O and LSE from one forward call made here
+    (outside any timed region) and a seeded upstream gradient dO."""
+    layout, P, cu = w["layout"], w["P"], w["cu"]
+    if layout not in ("contiguous", "zigzag", "striped"):
+        raise SystemExit(f"--pass bwd needs a ring workload, not {layout}")
+    qd, kd, vd = w["in"]
+    S, hq, hkv, dh = w["S"], w["hq"], w["hkv"], w["dh"]
+    if w["dtype"] != torch.bfloat16:
+        raise SystemExit("--pass bwd takes bf16 workloads")
+    do = synth.normal((S, hq, dh), synth.SEED_DO, 0.5)
+    if layout != "contiguous":
+        reorder = api.zigzag_reorder if layout == "zigzag" else api.striped_reorder
+        qd, kd, vd = (reorder(t, P) for t in (qd, kd, vd))
+        do = reorder(do.to(dev), P).cpu()
+    cu_dev = torch.tensor(cu, dtype=torch.int32, device=dev) if cu is not None else None
+    o, lse = w["out"]
+    api.ring_attn_fwd(qd, kd, vd, P, layout, True, cu, cu_dev, o=o, lse=lse, workspace=fwd_ws)
+    dod = do.to(dev)
+    dq = torch.empty((S, hq, dh), device=dev, dtype=torch.float32)
+    dk = torch.empty((S, hkv, dh), device=dev, dtype=torch.float32)
+    dv = torch.empty_like(dk)
+    ws = torch.empty(api.ring_attn_bwd_workspace_size(S, hq, hkv, dh, P, layout, True, cu), device=dev,
+                     dtype=torch.uint8)
+    torch.cuda.synchronize()
+
+    def step():
+        api.ring_attn_bwd(qd, kd, vd, o, lse, dod, P, layout, True, cu, cu_dev, dq=dq, dk=dk, dv=dv, workspace=ws)
+
     w["step"] = step
     w["ws_bytes"] = ws.numel()
-    return w
+    w["host"] = [t.cpu().pin_memory() for t in (qd, kd, vd, o, lse, dod)]
+    w["in"] = (qd, kd, vd, o, lse, dod)
+    w["out"] = (dq, dk, dv)
+    w["fwd_flops"] = w["flops"]
+    # five score-sized products (S, dP, dV, dK, dQ) against the forward's two
+    w["flops"] = 2.5 * w["flops"]
 
 
 def time_steps(w, steps, warmup, ws):
@@ -248,7 +293,11 @@ def time_steps(w, steps, warmup, ws):
     barrier(ws)
     total_ms = t0.elapsed_time(t1)
     attn_ms = [a.elapsed_time(b) for a, b in zip(ab, ae)]
-    merge_ms = [a.elapsed_time(b) for a, b in zip(ae, me)] if w["layout"] != "ulysses" else []
+    if w.get("pass") == "bwd":  # merge_end marks the boundary between the dQ and dK/dV kernels
+        merge_ms = {"dq": [a.elapsed_time(b) for a, b in zip(ab, me)],
+                    "dkdv": [a.elapsed_time(b) for a, b in zip(me, ae)]}
+    else:
+        merge_ms = [a.elapsed_time(b) for a, b in zip(ae, me)] if w["layout"] != "ulysses" else []
     err = api.device_error()
     if err:
         raise RuntimeError(f"device error word {err:#x}: a kernel gave up waiting")
@@ -256,21 +305,21 @@ def time_steps(w, steps, warmup, ws):
 
 
 def time_e2e(w, steps):
-    """Same step through the public API with host buffers: pinned host Q, K, V
-    copied in and O, LSE copied out inside the timed region."""
-    qh, kh, vh = w["host"]
-    qd, kd, vd = w["in"]
-    o, lse = w["out"]
-    oh = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
-    lh = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    """Same step through the public API with host buffers: the step's pinned
+    host inputs (Q, K, V; for the backward also O, LSE, dO) copied in and its
+    outputs (O, LSE; for the backward dQ, dK, dV) copied out inside the timed
+    region."""
+    hosts_in = w["host"]
+    devs_in = w["in"]
+    devs_out = w["out"]
+    hosts_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in devs_out]
 
     def one():
-        qd.copy_(qh, non_blocking=True)
-        kd.copy_(kh, non_blocking=True)
-        vd.copy_(vh, non_blocking=True)
+        for d, h in zip(devs_in, hosts_in):
+            d.copy_(h, non_blocking=True)
         w["step"]()
-        oh.copy_(o, non_blocking=True)
-        lh.copy_(lse, non_blocking=True)
+        for h, d in zip(hosts_out, devs_out):
+            h.copy_(d, non_blocking=True)
 
     one()
     torch.cuda.synchronize()
@@ -281,8 +330,8 @@ def time_e2e(w, steps):
     t1.record()
     torch.cuda.synchronize()
     ms = t0.elapsed_time(t1) / steps
-    h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
-    d2h = oh.numel() * oh.element_size() + lh.numel() * lh.element_size()
+    h2d = sum(t.numel() * t.element_size() for t in hosts_in)
+    d2h = sum(t.numel() * t.element_size() for t in hosts_out)
     return ms, h2d, d2h
 
 
@@ -323,7 +372,7 @@ def time_permute(reps=20):
 
 
 # ----------------------------------------------------------------- CPU oracle
-def oracle_sample_rate(w, target_s=12.0, max_rows=1024, seed=0):
+def oracle_sample_rate(w, target_s=12.0, max_rows=1024, seed=0, bwd=False):
     """Times the fp64 oracle on a bounded sample of the same workload: batches
     of 32 query rows (natural positions, seeded) against every key, all heads.
     Returns causal-effective TFLOP/s of the sample and what was sampled."""
@@ -333,24 +382,30 @@ def oracle_sample_rate(w, target_s=12.0, max_rows=1024, seed=0):
                                                                  std=w["cfg"]["std"], dtype=w["dtype"]))
     if w["dtype"] == torch.float32:  # the kernel consumes bf16-rounded values
         q, k, v = (torch.from_numpy(t).to(torch.bfloat16).double().numpy() for t in (q, k, v))
+    if bwd:
+        do = synth.normal((w["S"], w["hq"], w["dh"]), synth.SEED_DO, 0.5).double().numpy()
     rng = np.random.default_rng(seed)
     cu = w["cu"]
     t_total, flops, rows_done = 0.0, 0.0, 0
     while t_total < target_s and rows_done < max_rows:
         rows = np.sort(rng.integers(0, w["S"], 32))
         t0 = time.perf_counter()
-        ref.attention(q[rows], k, v, causal=True, cu_seqlens=cu, qpos=rows)
+        if bwd:  # the gradient work of these query rows (their dQ, their share of dK, dV)
+            ref.attention_bwd(q[rows], k, v, do[rows], causal=True, cu_seqlens=cu, qpos=rows)
+        else:
+            ref.attention(q[rows], k, v, causal=True, cu_seqlens=cu, qpos=rows)
         t_total += time.perf_counter() - t0
         if cu is None:
             live = (rows + 1).sum()
         else:
             starts = np.asarray(cu)[np.searchsorted(cu, rows, side="right") - 1]
             live = (rows - starts + 1).sum()
-        flops += 4.0 * w["dh"] * w["hq"] * float(live)
+        flops += (10.0 if bwd else 4.0) * w["dh"] * w["hq"] * float(live)
         rows_done += 32
     cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
     return dict(value=flops / t_total / 1e12, unit="TFLOP/s", cores=cores, kind="oracle",
-                sample=f"{rows_done} query rows (seeded, uniform positions) x all {w['S']} keys x {w['hq']} heads, "
+                sample=f"{'gradient of ' if bwd else ''}{rows_done} query rows (seeded, uniform positions) x all "
+                       f"{w['S']} keys x {w['hq']} heads, "
                        f"fp64 numpy, {t_total:.1f} s")
 
 
@@ -405,7 +460,8 @@ def run_ours(args, ws, rank, local):
     from context_exact_attention_step_b200 import build as _build
     _build.build()
     pk = peaks()
-    w = make_workload(args.workload, args.seq_len)
+    w = make_workload(args.workload, args.seq_len, args.pass_)
+    bwd = args.pass_ == "bwd"
     clocks = Clocks(local)
     clocks.start()
     total_ms, attn_ms, merge_ms, launches = time_steps(w, args.steps, args.warmup, ws)
@@ -418,10 +474,10 @@ def run_ours(args, ws, rank, local):
                                                       "attn_fwd.cu")), w["name"], w["S"]))
     e2e_ms, h2d, d2h = time_e2e(w, args.e2e_steps)
     e2e_ms = max_over_ranks(e2e_ms, ws)
-    perm = time_permute() if not args.no_permute else None
+    perm = time_permute() if not (args.no_permute or bwd) else None
     cfg = w["cfg"]
     line = {
-        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
+        "metric": METRIC_BWD if bwd else METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w["name"], "S": w["S"], "hq": w["hq"], "hkv": w["hkv"], "dh": w["dh"], "P": w["P"],
@@ -431,8 +487,10 @@ def run_ours(args, ws, rank, local):
                        sum(t.numel() * t.element_size() for t in w["in"]) / 1e6, w["ws_bytes"] / 1e6),
                    "per_gpu": "independent problem per GPU",
                    **({k_: cfg[k_] for k_ in ("Pr", "Pu", "ring_layout")} if w["layout"] == "usp" else {})},
-        "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel", "achieved": attn_tf, "peak": pk["bf16"],
-                     "unit": "TFLOP/s", "frac": attn_tf / pk["bf16"], "traffic": traffic,
+        "roofline": {"bound": "tensor",
+                     "kernel": "attn_bwd_dq_kernel + attn_bwd_dkdv_kernel" if bwd else "attn_fwd_kernel",
+                     "achieved": attn_tf, "peak": pk["bf16"],
+                     "unit": "TFLOP/s", "frac": attn_tf / pk["bf16"], "traffic": None if bwd else traffic,
                      "peak_source": pk["source"] + " burst bf16", "frac_of_sustained": attn_tf / pk["bf16_sus"],
                      "frac_of_nominal_2250": attn_tf / 2250.0, "attn_ms": attn_avg},
         "e2e": {"value": w["flops"] * ws / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
@@ -440,7 +498,16 @@ def run_ours(args, ws, rank, local):
         "gpu_launches": int(launches),
         "clocks": ck,
     }
-    if merge_ms:
+    if bwd:
+        # per kernel: time and the tensor work each one executes (dQ side: S,
+        # dP, dQ; dK/dV side: S^T, dP^T, dV, dK; two FLOP per multiply-add)
+        for name, gemms in (("dq", 3), ("dkdv", 4)):
+            kms = statistics.mean(merge_ms[name])
+            ex = gemms / 2.0 * w["fwd_flops"]
+            line["bwd_" + name] = {"ms": kms, "executed_tflops": ex / (kms * 1e-3) / 1e12,
+                                   "executed_frac": ex / (kms * 1e-3) / 1e12 / pk["bf16"]}
+        line["config"]["pass"] = "backward (prep + dQ kernel + dK/dV kernel), inputs in shard order"
+    elif merge_ms:
         mb = merge_bytes(w)
         mms = statistics.mean(merge_ms)
         line["merge"] = {"ms": mms, "gbs": mb / (mms * 1e-3) / 1e9, "frac_hbm": mb / (mms * 1e-3) / 1e9 / pk["hbm_gbs"],
@@ -449,7 +516,7 @@ def run_ours(args, ws, rank, local):
         line["a2a_permute"] = {"gbs": perm["gbs"], "frac_hbm": perm["gbs"] / pk["hbm_gbs"], "ms": perm["ms"],
                                "bytes": perm["bytes"], "workload": "ulysses_gqa_128k Q,K,V seq->head + fp32 O head->seq"}
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = oracle_sample_rate(w)
+        line["cpu_baseline"] = oracle_sample_rate(w, bwd=bwd)
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -477,6 +544,8 @@ def main():
     ap.add_argument("--workload", default="ring_contig_32k")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-permute", action="store_true")
+    ap.add_argument("--pass", dest="pass_", default="fwd", choices=["fwd", "bwd"],
+                    help="bwd: time the ring backward (dQ, dK, dV) of a ring workload instead of the forward")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seq-len", type=int, default=None,
                     help="override the workload's sequence length (smaller cases for profiler captures)")

@@ -832,6 +832,7 @@ cp_status cp_ring_attn_bwd(const void* q, const void* k, const void* v, const fl
       e = launch_bwd(dh, tq, tdo, tk, tv, plan, dq_side, st);
       if (e != cudaSuccess) return cuda_fail(e, dq_side ? "backward dQ launch" : "backward dK/dV launch");
     }
+    if (dq_side) record(g_ev_merge_end, st);
   }
   record(g_ev_attn_end, st);
   return ok();

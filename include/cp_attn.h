@@ -350,10 +350,13 @@ cp_status cp_ring_attn_fwd_noalloc(const void* q, const void* k, const void* v, 
 cp_status cp_kernel_launch_count(uint64_t* count);
 
 /* Profiling hook: when non-NULL, the composite calls (cp_ring_attn_fwd,
- * cp_ulysses_attn_fwd) made afterwards on the calling thread record
- * `attn_begin` / `attn_end` (cudaEvent_t passed as void*) on their stream
- * immediately before their first and after their last block-attention launch,
- * and `merge_end` after their last merge launch.  Pass NULLs to turn it off. */
+ * cp_ulysses_attn_fwd, cp_usp_attn_fwd) made afterwards on the calling thread
+ * record `attn_begin` / `attn_end` (cudaEvent_t passed as void*) on their
+ * stream immediately before their first and after their last block-attention
+ * launch, and `merge_end` after their last merge launch.  cp_ring_attn_bwd
+ * records `attn_begin` before its dQ kernel, `merge_end` between the dQ and
+ * the dK/dV kernels, and `attn_end` after the dK/dV kernel.  Pass NULLs to
+ * turn it off. */
 cp_status cp_set_profile_events(void* attn_begin, void* attn_end, void* merge_end);
 
 #ifdef __cplusplus

@@ -26,11 +26,13 @@
 //     head of the group, and accumulates dK and dV in tensor memory.
 // No atomics: every output row is written once by one CTA.
 //
-// CTA layout of both tensor-core kernels (256 threads, one CTA per SM):
+// CTA layout of both tensor-core kernels (384 threads, one CTA per SM):
 //   warp 0      TMA producer
 //   warp 1      tcgen05.mma issuer (one elected lane) and TMEM owner
 //   warps 2-3   idle
-//   warps 4-7   element-wise stage, one own row per thread (TMEM lane)
+//   warps 4-7   element-wise stage, columns 0-63 of every tile, one own row
+//               per thread (TMEM lane)
+//   warps 8-11  element-wise stage, columns 64-127 of the same rows
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -47,7 +49,7 @@ std::atomic<uint64_t>& launch_counter();
 
 namespace {
 
-constexpr int kBwdThreads = 256;
+constexpr int kBwdThreads = 384;
 constexpr int kNoLo = -(1 << 30);
 constexpr int kNoHi = (1 << 30);
 constexpr float kLog2e = 1.4426950408889634f;
@@ -192,8 +194,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     mbar_init(bar(B_S), 1);
     mbar_init(bar(B_DP), 1);
-    mbar_init(bar(B_SC), 4);  // one arrive per element-wise warp
-    mbar_init(bar(B_DS), 4);
+    mbar_init(bar(B_SC), 8);  // one arrive per element-wise warp
+    mbar_init(bar(B_DS), 8);
     mbar_init(bar(B_ACC), 1);
     mbar_init(bar(B_DRAIN), 1);
     *abort_flag = 0;
@@ -220,6 +222,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   decode_own(plan, plan.items[blockIdx.x / plan.hq], own);
   auto col_d = [](int j) { return (j & 1) ? C::kColD1 : C::kColD0; };
 
+  // Registers: launched at 168 per thread (384 threads); inside its own
+  // branch the control warpgroup (warps 0-3) drops to 64 and the two
+  // element-wise warpgroups rise to 216: 128 * 64 + 256 * 216 <= 384 * 168.
+  if (warp < 4) {
+    regs_dec<64>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     mbar_arrive_expect_tx_elect(bar(B_QD), 2 * T::kTileBytes);
@@ -265,12 +272,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_mma_ss_elect(tmem + dcol, a, b, idesc_ss, kk > 0 ? 1u : 0u);
       }
     };
-    // dQ += dS K: A = dS (bf16 in TMEM, 128 keys), B = the K tile read MN-major
-    auto issue_dq = [&](uint32_t acol, uint32_t kbase, bool acc) {
+    // dQ += dS K: A = dS (bf16 in TMEM, 128 keys as 8 K-steps of 16; keys
+    // 0-63 at dcol, keys 64-127 at dcol + 64), B = the K tile read MN-major
+    auto issue_dq = [&](uint32_t dcol, uint32_t kbase, bool acc) {
 #pragma unroll
       for (int kk = 0; kk < 128 / 16; ++kk) {
+        const uint32_t acol = kk < 4 ? dcol + kk * 8 : dcol + 64 + (kk - 4) * 8;
         const uint64_t b = sdesc_sw128(kbase + kk * 2048, T::kBoxBytes, 1024);
-        tc_mma_ts_elect(tmem + C::kColQ, tmem + acol + kk * 8, b, idesc_dq, (acc || kk > 0) ? 1u : 0u);
+        tc_mma_ts_elect(tmem + C::kColQ, tmem + acol, b, idesc_dq, (acc || kk > 0) ? 1u : 0u);
       }
     };
     auto kslot = [&](int j) { return (2 * j) % C::kStages; };
@@ -329,8 +338,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     tc_commit_elect(bar(B_ACC));
     tc_commit_elect(bar(B_DRAIN));
     mbar_wait_warp(bar(B_DRAIN), 0, abort_flag, nullptr, 1000000000ull);
-  } else if (warp >= 4) {
+  }
+  } else {
+    regs_inc<216>();
     // ------------------------------------------------------------ element-wise
+    // Two warpgroups share each query row (TMEM lane): warpgroup hh owns key
+    // columns [64 hh, 64 hh + 64) of every tile, so two warps per scheduler
+    // hide each other's latency.  dS is written over dP columns the same
+    // warpgroup has read: hh = 0 -> [0, 32), hh = 1 -> [64, 96).
+    const int hh = (warp - 4) >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
@@ -346,6 +362,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint64_t c2 = f2_pack(plan.scale_log2, plan.scale_log2);
     const uint64_t nl2 = f2_pack(neg_lg, neg_lg);
     const uint64_t nd2 = f2_pack(-dd, -dd);
+    const int c0 = hh * 64;
+    const uint32_t ds_off = hh ? 64u : 0u;
     DqIter it;
     it.init(plan, own);
     KvTile kt;
@@ -356,26 +374,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      uint32_t s[128];
-      const uint32_t tS = tmem + lane_base + C::kColS;
+      uint32_t s[64];
+      const uint32_t tS = tmem + lane_base + C::kColS + c0;
       tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
       tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
-      tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
-      tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
       tc_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(B_SC));
       if (!kt.full) {
-        const int clo = row_lo - kt.pos;
-        const int chi = min(row_hi - kt.pos, kt.valid - 1);
+        const int clo = row_lo - kt.pos - c0;
+        const int chi = min(row_hi - kt.pos, kt.valid - 1) - c0;
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
+        for (int c = 0; c < 64; ++c)
           if (c < clo || c > chi) s[c] = __float_as_uint(-CUDART_INF_F);
       }
       // P = 2^(S * scale * log2(e) - LSE * log2(e)), in place
 #pragma unroll
-      for (int c = 0; c < 128; c += 2) {
+      for (int c = 0; c < 64; c += 2) {
         float x0, x1;
         f2_unpack(f2_fma(f2_pack(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), c2, nl2), x0, x1);
         s[c] = __float_as_uint(ex2_approx(x0));
@@ -386,23 +402,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const uint32_t tD = tmem + lane_base + col_d(j);
+      uint32_t w[32];
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
+      for (int ch = 0; ch < 2; ++ch) {
         uint32_t d[32];
-        tmem_ld32(tD + ch * 32, d);
+        tmem_ld32(tD + c0 + ch * 32, d);
         tc_wait_ld();
-        uint32_t w[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int c = ch * 32 + 2 * i;
           const uint64_t t = f2_add(f2_pack(__uint_as_float(d[2 * i]), __uint_as_float(d[2 * i + 1])), nd2);
           float a, b;
           f2_unpack(f2_mul(f2_pack(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), t), a, b);
-          w[i] = pack_bf16x2(a, b);
+          w[ch * 16 + i] = pack_bf16x2(a, b);
         }
-        // columns [16 ch, 16 ch + 16) of this buffer have already been read
-        tmem_st16(tD + ch * 16, w);
       }
+      tmem_st32(tD + ds_off, w);
       tc_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -414,13 +429,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
     }
     if (ok) {
+      // warpgroup hh writes dQ columns [hh DH/2, (hh + 1) DH/2)
       tc_fence_after();
-      float* dst = plan.dq + ((size_t)(own.buf_row0 + row) * plan.hq + h) * DH;
+      float* dst = plan.dq + ((size_t)(own.buf_row0 + row) * plan.hq + h) * DH + hh * (DH / 2);
 #pragma unroll 1
-      for (int ch = 0; ch < DH / 32; ++ch) {
+      for (int ch = 0; ch < DH / 64; ++ch) {
         uint32_t o[32];
         if (j > 0) {
-          tmem_ld32(tmem + lane_base + C::kColQ + ch * 32, o);
+          tmem_ld32(tmem + lane_base + C::kColQ + hh * (DH / 2) + ch * 32, o);
           tc_wait_ld();
         }
         if (rvalid) {
@@ -438,7 +454,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
     }
   }
-
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -568,8 +583,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     mbar_init(bar(B_S), 1);
     mbar_init(bar(B_DP), 1);
-    mbar_init(bar(B_P), 4);
-    mbar_init(bar(B_DS), 4);
+    mbar_init(bar(B_P), 8);  // one arrive per element-wise warp
+    mbar_init(bar(B_DS), 8);
     mbar_init(bar(B_ACC), 1);
     mbar_init(bar(B_DRAIN), 1);
     *abort_flag = 0;
@@ -597,6 +612,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   auto stage_q = [&](int s) { return sStage + s * C::kStageBytes; };
   auto stage_do = [&](int s) { return sStage + s * C::kStageBytes + T::kTileBytes; };
 
+  // Registers: launched at 168 per thread (384 threads); inside its own
+  // branch the control warpgroup (warps 0-3) drops to 64 and the two
+  // element-wise warpgroups rise to 216: 128 * 64 + 256 * 216 <= 384 * 168.
+  if (warp < 4) {
+    regs_dec<64>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     mbar_arrive_expect_tx_elect(bar(B_KV), 2 * T::kTileBytes);
@@ -609,7 +629,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     QTile qt;
     uint32_t c = 0;
     bool ok = true;
-    while (ok && it.next(qt)) {
+    // -LSE*log2(e) and D of a tile's query rows (0 past the tile's end).  The
+    // loads for the next tile are issued as soon as the current tile's values
+    // are stored, so their latency hides behind the wait for a free stage.
+    float nl[4], nd[4];
+    auto load_vec = [&](const QTile& x) {
+      const size_t base = (size_t)x.h * plan.S + x.buf_row;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int cidx = lane + 32 * i;
+        const bool in = cidx < x.valid;
+        nl[i] = in ? -__ldg(plan.lg + base + cidx) : 0.f;
+        nd[i] = in ? __ldg(plan.dd + base + cidx) : 0.f;
+      }
+    };
+    bool have = it.next(qt);
+    if (have) load_vec(qt);
+    while (ok && have) {
       const int slot = c % C::kStages;
       const uint32_t ph = (c / C::kStages) & 1u;
       ok = mbar_wait_warp(bar(B_EMPTY + slot), ph ^ 1u, abort_flag, err, kWaitNs);
@@ -621,18 +657,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tma_load_2d_elect(smem_addr(stage_do(slot) + b * T::kBoxBytes), &tm_do, qt.h * DH + b * 64, qt.buf_row,
                           bar(B_FULL + slot));
       }
-      // -LSE*log2(e) and D of the tile's query rows (0 past the tile's end)
       float* vl = sVec + slot * (C::kVecBytes / 4);
       float* vd = vl + 128;
-      const size_t base = (size_t)qt.h * plan.S + qt.buf_row;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const int cidx = lane + 32 * i;
-        const bool in = cidx < qt.valid;
-        vl[cidx] = in ? -__ldg(plan.lg + base + cidx) : 0.f;
-        vd[cidx] = in ? __ldg(plan.dd + base + cidx) : 0.f;
+        vl[lane + 32 * i] = nl[i];
+        vd[lane + 32 * i] = nd[i];
       }
+      QTile nx;
+      have = it.next(nx);
+      if (have) load_vec(nx);
       mbar_arrive(bar(B_FULL + slot));  // release: the stores above are visible to the waiters
+      qt = nx;
       ++c;
     }
     const uint32_t first = c > (uint32_t)C::kStages ? c - C::kStages : 0u;
@@ -653,13 +689,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_mma_ss_elect(tmem + dcol, a, b, idesc_ss, kk > 0 ? 1u : 0u);
       }
     };
-    // D[dcol] += A (bf16 in TMEM at acol, 128 query rows) x B (a 128-row
-    // query-side tile read MN-major)
-    auto issue_acc = [&](uint32_t dcol, uint32_t acol, uint32_t b_base, bool acc) {
+    // D[dcol] += A (bf16 in TMEM, 128 query rows as 8 K-steps of 16) x B (a
+    // 128-row query-side tile read MN-major).  The A columns of K-steps 0-3
+    // (queries 0-63) start at lo_col, those of K-steps 4-7 at hi_col.
+    auto issue_acc = [&](uint32_t dcol, uint32_t lo_col, uint32_t hi_col, uint32_t b_base, bool acc) {
 #pragma unroll
       for (int kk = 0; kk < 128 / 16; ++kk) {
+        const uint32_t acol = kk < 4 ? lo_col + kk * 8 : hi_col + (kk - 4) * 8;
         const uint64_t b = sdesc_sw128(b_base + kk * 2048, T::kBoxBytes, 1024);
-        tc_mma_ts_elect(tmem + dcol, tmem + acol + kk * 8, b, idesc_acc, (acc || kk > 0) ? 1u : 0u);
+        tc_mma_ts_elect(tmem + dcol, tmem + acol, b, idesc_acc, (acc || kk > 0) ? 1u : 0u);
       }
     };
     auto slot_of = [&](int i) { return i % C::kStages; };
@@ -687,7 +725,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int s = slot_of(i);
       if (!(ok = mbar_wait_warp(bar(B_P), i & 1u, abort_flag, err, kWaitNs))) break;
       tc_fence_after();
-      issue_acc(C::kColDV, col_r(i), smem_addr(stage_do(s)), i > 0);
+      issue_acc(C::kColDV, col_r(i) + 0, col_r(i) + 96, smem_addr(stage_do(s)), i > 0);
       if (!(ok = mbar_wait_warp(bar(B_DS), i & 1u, abort_flag, err, kWaitNs))) break;
       tc_fence_after();
       if (hn) {
@@ -696,7 +734,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         issue_ss(col_r(i + 1), sk, smem_addr(stage_q(slot_of(i + 1))));
         tc_commit_elect(bar(B_S));
       }
-      issue_acc(C::kColDK, col_r(i) + 64, smem_addr(stage_q(s)), i > 0);
+      issue_acc(C::kColDK, col_r(i) + 32, col_r(i) + 64, smem_addr(stage_q(s)), i > 0);
       tc_commit_elect(bar(B_EMPTY + s));
       if (hn) {
         // dP^T(i+1) goes where P^T(i) / dS^T(i) live: issued after the two
@@ -711,8 +749,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     tc_commit_elect(bar(B_ACC));
     tc_commit_elect(bar(B_DRAIN));
     mbar_wait_warp(bar(B_DRAIN), 0, abort_flag, nullptr, 1000000000ull);
-  } else if (warp >= 4) {
+  }
+  } else {
+    regs_inc<216>();
     // ------------------------------------------------------------ element-wise
+    // Two warpgroups share each key row (TMEM lane): warpgroup hh owns query
+    // columns [64 hh, 64 hh + 64) of every tile, so two warps per scheduler
+    // hide each other's latency.  Each writes its packed P^T and dS^T only
+    // over S^T columns it has itself read:
+    //   hh = 0: P^T(q 0-63) -> cols [0, 32),   dS^T(q 0-63) -> cols [32, 64)
+    //   hh = 1: dS^T(q 64-127) -> cols [64, 96), P^T(q 64-127) -> cols [96, 128)
+    const int hh = (warp - 4) >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
@@ -724,6 +771,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                            : kNoHi;
     const int col_hi = rvalid ? (docs ? bdoc_last(plan.cu_seqlens, plan.n_docs, kpos) : kNoHi) : kNoLo;
     const uint64_t c2 = f2_pack(plan.scale_log2, plan.scale_log2);
+    const int c0 = hh * 64;                    // first query column of this warpgroup
+    const uint32_t p_col = hh ? 96u : 0u;      // where its P^T goes
+    const uint32_t ds_col = hh ? 64u : 32u;    // where its dS^T goes
     KvIter it;
     it.init(plan, own, hk);
     QTile qt;
@@ -731,45 +781,44 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     bool ok = true;
     while (it.next(qt)) {
       const int s = i % C::kStages;
-      const float* vl = sVec + s * (C::kVecBytes / 4);
-      const float* vd = vl + 128;
+      const float* vl = sVec + s * (C::kVecBytes / 4) + c0;
+      const float* vd = sVec + s * (C::kVecBytes / 4) + 128 + c0;
       ok = mbar_wait(bar(B_S), i & 1u, abort_flag, err, kWaitNs);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
       // P^T = 2^(S^T * scale * log2(e) - LSE_q * log2(e)), kept only as the
-      // bf16 pairs the dV MMA reads: S^T is read in two 64-column halves and
-      // P^T of half h is stored over columns [32 h, 32 h + 32), which hold S^T
-      // values already read.
+      // bf16 pairs the dV MMA reads
       const uint32_t tR = tmem + lane_base + col_r(i);
       const int shift = (plan.striped && plan.causal && own.rank > qt.r && rvalid) ? 1 : 0;
-      const int clo = lo0 + shift - qt.pos;
-      const int chi = min(col_hi - qt.pos, qt.valid - 1);
-      uint32_t pk[64];
-#pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
+      const int clo = lo0 + shift - qt.pos - c0;
+      const int chi = min(col_hi - qt.pos, qt.valid - 1) - c0;
+      uint32_t pk[32];
+      {
         uint32_t sv[64];
-        tmem_ld32(tR + h2 * 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-        tmem_ld32(tR + h2 * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+        tmem_ld32(tR + c0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+        tmem_ld32(tR + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
         tc_wait_ld();
         if (!qt.full) {
 #pragma unroll
-          for (int cc = 0; cc < 64; ++cc) {
-            const int c = h2 * 64 + cc;
-            if (c < clo || c > chi) sv[cc] = __float_as_uint(-CUDART_INF_F);
-          }
+          for (int cc = 0; cc < 64; ++cc)
+            if (cc < clo || cc > chi) sv[cc] = __float_as_uint(-CUDART_INF_F);
         }
 #pragma unroll
-        for (int i2 = 0; i2 < 32; ++i2) {
-          const float2 l2 = *reinterpret_cast<const float2*>(vl + h2 * 64 + 2 * i2);
-          float x0, x1;
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[2 * i2]), __uint_as_float(sv[2 * i2 + 1])), c2,
-                           f2_pack(l2.x, l2.y)),
+        for (int i4 = 0; i4 < 16; ++i4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(vl + 4 * i4);
+          float x0, x1, x2, x3;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[4 * i4]), __uint_as_float(sv[4 * i4 + 1])), c2,
+                           f2_pack(l4.x, l4.y)),
                     x0, x1);
-          pk[h2 * 32 + i2] = pack_bf16x2(ex2_approx(x0), ex2_approx(x1));
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[4 * i4 + 2]), __uint_as_float(sv[4 * i4 + 3])), c2,
+                           f2_pack(l4.z, l4.w)),
+                    x2, x3);
+          pk[2 * i4] = pack_bf16x2(ex2_approx(x0), ex2_approx(x1));
+          pk[2 * i4 + 1] = pack_bf16x2(ex2_approx(x2), ex2_approx(x3));
         }
-        tmem_st32(tR + h2 * 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[h2 * 32]));
       }
+      tmem_st32(tR + p_col, pk);
       tc_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -778,26 +827,29 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      // dS^T = P^T * (dP^T - D_q) from the bf16 P^T, over columns [64, 128)
-      const uint32_t tD = tmem + lane_base + col_r(i + 1);
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t d[32];
-        tmem_ld32(tD + ch * 32, d);
+      // dS^T = P^T * (dP^T - D_q) from the bf16 P^T
+      {
+        const uint32_t tD = tmem + lane_base + col_r(i + 1) + c0;
+        uint32_t d[64];
+        tmem_ld32(tD, *reinterpret_cast<uint32_t(*)[32]>(&d[0]));
+        tmem_ld32(tD + 32, *reinterpret_cast<uint32_t(*)[32]>(&d[32]));
         tc_wait_ld();
-        uint32_t w[16];
+        uint32_t w[32];
 #pragma unroll
-        for (int i2 = 0; i2 < 16; ++i2) {
-          const int c = ch * 32 + 2 * i2;
-          const uint32_t pw = pk[ch * 16 + i2];
-          const float2 d2 = *reinterpret_cast<const float2*>(vd + c);
-          const uint64_t t = f2_add(f2_pack(__uint_as_float(d[2 * i2]), __uint_as_float(d[2 * i2 + 1])),
-                                    f2_pack(-d2.x, -d2.y));
-          float a, b;
-          f2_unpack(f2_mul(f2_pack(__uint_as_float(pw << 16), __uint_as_float(pw & 0xFFFF0000u)), t), a, b);
-          w[i2] = pack_bf16x2(a, b);
+        for (int i4 = 0; i4 < 16; ++i4) {
+          const float4 d4 = *reinterpret_cast<const float4*>(vd + 4 * i4);
+          const uint32_t pw0 = pk[2 * i4], pw1 = pk[2 * i4 + 1];
+          const uint64_t t0 = f2_add(f2_pack(__uint_as_float(d[4 * i4]), __uint_as_float(d[4 * i4 + 1])),
+                                     f2_pack(-d4.x, -d4.y));
+          const uint64_t t1 = f2_add(f2_pack(__uint_as_float(d[4 * i4 + 2]), __uint_as_float(d[4 * i4 + 3])),
+                                     f2_pack(-d4.z, -d4.w));
+          float a0, a1, a2, a3;
+          f2_unpack(f2_mul(f2_pack(__uint_as_float(pw0 << 16), __uint_as_float(pw0 & 0xFFFF0000u)), t0), a0, a1);
+          f2_unpack(f2_mul(f2_pack(__uint_as_float(pw1 << 16), __uint_as_float(pw1 & 0xFFFF0000u)), t1), a2, a3);
+          w[2 * i4] = pack_bf16x2(a0, a1);
+          w[2 * i4 + 1] = pack_bf16x2(a2, a3);
         }
-        tmem_st16(tR + 64 + ch * 16, w);
+        tmem_st32(tR + ds_col, w);
       }
       tc_wait_st();
       tc_fence_before();
@@ -810,37 +862,34 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
     }
     if (ok) {
+      // warpgroup 0 writes dV, warpgroup 1 writes dK * scale
       tc_fence_after();
       const size_t orow = (size_t)(own.buf_row0 + row) * plan.hkv + hk;
+      float* dst = (hh == 0 ? plan.dv : plan.dk) + orow * DH;
+      const uint32_t col = hh == 0 ? C::kColDV : C::kColDK;
+      const float f = hh == 0 ? 1.f : plan.scale;
 #pragma unroll 1
-      for (int which = 0; which < 2; ++which) {
-        float* dst = (which == 0 ? plan.dv : plan.dk) + orow * DH;
-        const uint32_t col = which == 0 ? C::kColDV : C::kColDK;
-        const float f = which == 0 ? 1.f : plan.scale;
-#pragma unroll 1
-        for (int ch = 0; ch < DH / 32; ++ch) {
-          uint32_t o[32];
-          if (i > 0) {
-            tmem_ld32(tmem + lane_base + col + ch * 32, o);
-            tc_wait_ld();
-          }
-          if (rvalid) {
-            float4* d4 = reinterpret_cast<float4*>(dst + ch * 32);
+      for (int ch = 0; ch < DH / 32; ++ch) {
+        uint32_t o[32];
+        if (i > 0) {
+          tmem_ld32(tmem + lane_base + col + ch * 32, o);
+          tc_wait_ld();
+        }
+        if (rvalid) {
+          float4* d4 = reinterpret_cast<float4*>(dst + ch * 32);
 #pragma unroll
-            for (int k4 = 0; k4 < 8; ++k4) {
-              float4 v;
-              v.x = i > 0 ? __uint_as_float(o[4 * k4 + 0]) * f : 0.f;
-              v.y = i > 0 ? __uint_as_float(o[4 * k4 + 1]) * f : 0.f;
-              v.z = i > 0 ? __uint_as_float(o[4 * k4 + 2]) * f : 0.f;
-              v.w = i > 0 ? __uint_as_float(o[4 * k4 + 3]) * f : 0.f;
-              d4[k4] = v;
-            }
+          for (int k4 = 0; k4 < 8; ++k4) {
+            float4 v;
+            v.x = i > 0 ? __uint_as_float(o[4 * k4 + 0]) * f : 0.f;
+            v.y = i > 0 ? __uint_as_float(o[4 * k4 + 1]) * f : 0.f;
+            v.z = i > 0 ? __uint_as_float(o[4 * k4 + 2]) * f : 0.f;
+            v.w = i > 0 ? __uint_as_float(o[4 * k4 + 3]) * f : 0.f;
+            d4[k4] = v;
           }
         }
       }
     }
   }
-
   tc_fence_before();
   __syncthreads();
   tc_fence_after();

@@ -123,6 +123,33 @@ def test_usp_workspace_is_copies_plus_pu_rings(layout):
     assert api.usp_attn_workspace_size(S, hq, hkv, dh, Pr, Pu, layout) == want
 
 
+def _bwd(S=1024, hq=4, hkv=4, dh=128, P=4, layout=_lib.CP_LAYOUT_ZIGZAG, ws=FAKE, wsb=1 << 40, dq=FAKE,
+         dout=FAKE, cu=None, n_docs=0):
+    return lib().cp_ring_attn_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, dout, S, hq, hkv, dh, P, layout, _lib.CP_MASK_CAUSAL,
+                                  cu, ctypes.c_void_p(0) if not n_docs else FAKE, n_docs, 0.0, dq, FAKE, FAKE, ws,
+                                  wsb, ctypes.c_void_p(0))
+
+
+def test_ring_bwd_rejects_bad_arguments():
+    assert _bwd(dh=96) == _lib.CP_ERR_UNSUPPORTED
+    assert _bwd(hq=6, hkv=4) == _lib.CP_ERR_INVALID_ARG
+    assert _bwd(S=1028) == _lib.CP_ERR_INVALID_ARG                   # 2P does not divide S (zigzag)
+    assert _bwd(P=17) == _lib.CP_ERR_UNSUPPORTED
+    assert _bwd(dq=ctypes.c_void_p(0)) == _lib.CP_ERR_INVALID_ARG
+    assert _bwd(dout=MISALIGNED) == _lib.CP_ERR_ALIGNMENT
+    assert _bwd(ws=ctypes.c_void_p(0), wsb=0) == _lib.CP_ERR_WORKSPACE
+    assert _bwd(wsb=1024) == _lib.CP_ERR_WORKSPACE
+    cu = (ctypes.c_int32 * 3)(0, 600, 1024)
+    assert _bwd(layout=_lib.CP_LAYOUT_STRIPED, cu=cu, n_docs=2) == _lib.CP_ERR_UNSUPPORTED
+    assert len(lib().cp_last_error_string()) > 0
+
+
+def test_ring_bwd_workspace_is_two_vectors_per_head():
+    # D and LSE*log2(e), fp32 [hq][S] each, 256-byte aligned
+    a = lambda x: (x + 255) // 256 * 256
+    assert api.ring_attn_bwd_workspace_size(4096, 32, 8, 128, 4, "zigzag") == 2 * a(4096 * 32 * 4)
+
+
 def test_permute_and_merge_reject_bad_arguments():
     L = lib()
     # Ulysses head limit: P must divide the head count

@@ -19,9 +19,11 @@ from .api import (  # noqa: F401
     ring_attn_fwd,
     ring_attn_workspace_size,
     ring_schedule,
+    ulysses_attn_bwd,
     ulysses_attn_fwd,
     ulysses_attn_workspace_size,
     ulysses_permute,
+    usp_attn_bwd,
     usp_attn_fwd,
     usp_attn_workspace_size,
     zigzag_reorder,

@@ -26,6 +26,7 @@ EXPORTS = [
     "cp_device_error", "cp_kernel_launch_count", "cp_set_profile_events",
     "cp_ring_attn_fwd_noalloc", "cp_selftest_wait_timeout", "cp_striped_reorder",
     "cp_usp_attn_workspace_size", "cp_usp_attn_fwd", "cp_ring_attn_bwd_workspace_size", "cp_ring_attn_bwd",
+    "cp_usp_attn_bwd_workspace_size", "cp_usp_attn_bwd", "cp_ulysses_attn_bwd_workspace_size", "cp_ulysses_attn_bwd",
 ]
 
 
@@ -95,6 +96,17 @@ def lib():
     L.cp_ring_attn_bwd.restype = i32
     L.cp_ring_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, P32, vp, i32, f32,
                                    vp, vp, vp, vp, ctypes.c_size_t, vp]
+    L.cp_usp_attn_bwd_workspace_size.restype = i32
+    L.cp_usp_attn_bwd_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, P32, i32,
+                                                 ctypes.POINTER(ctypes.c_size_t)]
+    L.cp_usp_attn_bwd.restype = i32
+    L.cp_usp_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, P32, vp, i32, f32,
+                                  vp, vp, vp, vp, ctypes.c_size_t, vp]
+    L.cp_ulysses_attn_bwd_workspace_size.restype = i32
+    L.cp_ulysses_attn_bwd_workspace_size.argtypes = [i32, i32, i32, i32, i32, ctypes.POINTER(ctypes.c_size_t)]
+    L.cp_ulysses_attn_bwd.restype = i32
+    L.cp_ulysses_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp, vp, vp, vp,
+                                      ctypes.c_size_t, vp]
     L.cp_ring_schedule.restype = i32
     L.cp_ring_schedule.argtypes = [i32, i32, i32, i32, P32, i32, P32, P32, P32, P64]
     L.cp_count_live_pairs.restype = i32

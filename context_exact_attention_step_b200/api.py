@@ -329,6 +329,66 @@ def ring_attn_bwd(q, k, v, o, lse, do, P, layout="contiguous", causal=True, cu_s
     return dq, dk, dv
 
 
+def _bwd_outputs(q, k, dq, dk, dv):
+    S, hq, dh = q.shape
+    hkv = k.shape[1]
+    if dq is None:
+        dq = torch.empty((S, hq, dh), device=q.device, dtype=torch.float32)
+    if dk is None:
+        dk = torch.empty((S, hkv, dh), device=q.device, dtype=torch.float32)
+    if dv is None:
+        dv = torch.empty((S, hkv, dh), device=q.device, dtype=torch.float32)
+    return dq, dk, dv
+
+
+def _bwd_check(q, k, v, o, lse, do):
+    for n, t in (("q", q), ("k", k), ("v", v), ("do", do)):
+        _need_cuda(n, t, torch.bfloat16)
+    _need_cuda("o", o, torch.float32)
+    _need_cuda("lse", lse, torch.float32)
+
+
+def usp_attn_bwd(q, k, v, o, lse, do, Pr, Pu, layout="contiguous", causal=True, cu_seqlens=None,
+                 cu_seqlens_dev=None, softmax_scale=0.0, dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """Gradients of usp_attn_fwd: tensors as for ring_attn_bwd, in the
+    forward's storage order (``layout`` over Pr ring groups)."""
+    _bwd_check(q, k, v, o, lse, do)
+    S, hq, dh = q.shape
+    hkv = k.shape[1]
+    cu_p, n_docs, cu_np = _cu_host(cu_seqlens)
+    if n_docs > 0 and cu_seqlens_dev is None:
+        cu_seqlens_dev = torch.from_numpy(cu_np).to(q.device)
+    dq, dk, dv = _bwd_outputs(q, k, dq, dk, dv)
+    if workspace is None:
+        out = ctypes.c_size_t(0)
+        check(lib().cp_usp_attn_bwd_workspace_size(S, hq, hkv, dh, Pr, Pu, _LAYOUTS[layout],
+                                                   _lib.CP_MASK_CAUSAL if causal else _lib.CP_MASK_NONE, cu_p,
+                                                   n_docs, ctypes.byref(out)))
+        workspace = torch.empty(max(int(out.value), 256), device=q.device, dtype=torch.uint8)
+    check(lib().cp_usp_attn_bwd(_vp(q), _vp(k), _vp(v), _vp(o), _vp(lse), _vp(do), S, hq, hkv, dh, Pr, Pu,
+                                _LAYOUTS[layout], _lib.CP_MASK_CAUSAL if causal else _lib.CP_MASK_NONE, cu_p,
+                                _vp(cu_seqlens_dev), n_docs, float(softmax_scale), _vp(dq), _vp(dk), _vp(dv),
+                                _vp(workspace), workspace.numel(), _stream(stream)))
+    return dq, dk, dv
+
+
+def ulysses_attn_bwd(q, k, v, o, lse, do, P, causal=True, softmax_scale=0.0, dq=None, dk=None, dv=None,
+                     workspace=None, stream=None):
+    """Gradients of ulysses_attn_fwd, tensors in natural sequence order."""
+    _bwd_check(q, k, v, o, lse, do)
+    S, hq, dh = q.shape
+    hkv = k.shape[1]
+    dq, dk, dv = _bwd_outputs(q, k, dq, dk, dv)
+    if workspace is None:
+        out = ctypes.c_size_t(0)
+        check(lib().cp_ulysses_attn_bwd_workspace_size(S, hq, hkv, dh, P, ctypes.byref(out)))
+        workspace = torch.empty(max(int(out.value), 256), device=q.device, dtype=torch.uint8)
+    check(lib().cp_ulysses_attn_bwd(_vp(q), _vp(k), _vp(v), _vp(o), _vp(lse), _vp(do), S, hq, hkv, dh, P,
+                                    _lib.CP_MASK_CAUSAL if causal else _lib.CP_MASK_NONE, float(softmax_scale),
+                                    _vp(dq), _vp(dk), _vp(dv), _vp(workspace), workspace.numel(), _stream(stream)))
+    return dq, dk, dv
+
+
 def ring_schedule(S, P, layout="contiguous", causal=True, cu_seqlens=None):
     """Host-only view of the ring-step schedule: arrays of P*P entries indexed
     r*P + t (see cp_ring_schedule)."""

@@ -31,8 +31,8 @@ cudaError_t launch_zigzag(const void* in, void* out, int P, int batch, size_t ch
 cudaError_t launch_f32_to_bf16(const float* in, void* out, size_t n, cudaStream_t st);
 cudaError_t launch_striped(const void* in, void* out, int P, int S, int batch, size_t row_bytes, int inverse,
                            cudaStream_t st);
-cudaError_t launch_bwd_prep(int dh, const float* o, const void* dout, const float* lse, int S, int hq, float* lg,
-                            float* dd, cudaStream_t st);
+cudaError_t launch_bwd_prep(int dh, const float* o, const void* dout, const float* lse, int G, int hg, int groups,
+                            float* lg, float* dd, cudaStream_t st);
 cudaError_t launch_bwd(int dh, const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
                        const CUtensorMap& tv, const cp_bwd_plan& plan, bool dq_side, cudaStream_t st);
 std::atomic<uint64_t>& launch_counter();
@@ -718,9 +718,9 @@ struct BwdItem {
   int64_t cost;
 };
 
-// Own 128-row tiles of every rank (dq_side) or shard, ordered by the number
-// of (q, k) pairs they admit, heaviest first.
-std::vector<uint32_t> bwd_items(const cp_bwd_plan& pl, bool dq_side, const Docs& docs) {
+// Own 128-row tiles of every rank (dq_side) or shard and every head group,
+// ordered by the number of (q, k) pairs they admit, heaviest first.
+std::vector<uint32_t> bwd_items(const cp_bwd_plan& pl, int groups, bool dq_side, const Docs& docs) {
   std::vector<BwdItem> v;
   for (int a = 0; a < pl.P; ++a)
     for (int sg = 0; sg < pl.nseg[a]; ++sg) {
@@ -740,7 +740,8 @@ std::vector<uint32_t> bwd_items(const cp_bwd_plan& pl, bool dq_side, const Docs&
               cost += count_admitted(other.pos, other.len, pos + shift, len, pl.causal != 0, docs);
             }
           }
-        v.push_back({((uint32_t)a << 24) | ((uint32_t)sg << 23) | (uint32_t)t, cost});
+        for (int g = 0; g < groups; ++g)
+          v.push_back({((uint32_t)a << 26) | ((uint32_t)sg << 25) | ((uint32_t)g << 19) | (uint32_t)t, cost});
       }
     }
   std::stable_sort(v.begin(), v.end(), [](const BwdItem& x, const BwdItem& y) { return x.cost > y.cost; });
@@ -749,39 +750,23 @@ std::vector<uint32_t> bwd_items(const cp_bwd_plan& pl, bool dq_side, const Docs&
   for (const BwdItem& x : v) out.push_back(x.code);
   return out;
 }
-}  // namespace
 
-cp_status cp_ring_attn_bwd(const void* q, const void* k, const void* v, const float* o, const float* lse,
-                           const void* dout, int S, int hq, int hkv, int dh, int P, cp_layout layout, cp_mask mask,
-                           const int32_t* cu_seqlens_host, const int32_t* cu_seqlens_dev, int n_docs,
-                           float softmax_scale, float* dq, float* dk, float* dv, void* workspace, size_t ws_bytes,
-                           void* stream) {
+// The ring backward over P ranks for `groups` blocks of heads.  qh, kh, vh,
+// doh are the head-major bf16 buffers ([groups][S][hg | hkg][dh]; one group:
+// the plain sharded buffers) the tensor cores read; dout, o, lse, dq, dk, dv
+// are in the final [S][groups * h][dh] / [groups * hq][S] layouts; lg, dd
+// are fp32 [hg][groups * S].
+cp_status run_bwd(const void* qh, const void* kh, const void* vh, const void* doh, const void* dout, const float* o,
+                  const float* lse, int S, int groups, int hg, int hkg, int dh, int P, cp_layout layout, cp_mask mask,
+                  const int32_t* cu_host, const int32_t* cu_dev, int n_docs, float softmax_scale, float* dq,
+                  float* dk, float* dv, float* lg, float* dd, cudaStream_t st) {
   cp_status s;
-  if ((s = ring_check(S, hq, hkv, dh, P, layout, mask, CP_BF16, cu_seqlens_host, n_docs)) != CP_OK) return s;
-  CP_CHECK_PTR(q);
-  CP_CHECK_PTR(k);
-  CP_CHECK_PTR(v);
-  CP_CHECK_PTR(o);
-  CP_CHECK_PTR(lse);
-  CP_CHECK_PTR(dout);
-  CP_CHECK_PTR(dq);
-  CP_CHECK_PTR(dk);
-  CP_CHECK_PTR(dv);
-  if (P > CP_BWD_MAX_RANKS) return fail(CP_ERR_UNSUPPORTED, "P = %d (backward supports 1..%d)", P, CP_BWD_MAX_RANKS);
-  if (n_docs > 0 && !cu_seqlens_dev) return fail(CP_ERR_INVALID_ARG, "n_docs > 0 needs cu_seqlens_dev");
-  const size_t need = bwd_workspace(S, hq);
-  if (!workspace || ws_bytes < need)
-    return fail(CP_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws_bytes);
-  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return fail(CP_ERR_ALIGNMENT, "workspace is not 256-byte aligned");
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  float* lg = static_cast<float*>(workspace);
-  float* dd = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + align256((size_t)S * hq * sizeof(float)));
-
+  const int64_t rows = (int64_t)groups * S;
   CUtensorMap tq, tdo, tk, tv;
-  if ((s = make_map(&tq, q, S, (int64_t)hq * dh, 128)) != CP_OK) return s;
-  if ((s = make_map(&tdo, dout, S, (int64_t)hq * dh, 128)) != CP_OK) return s;
-  if ((s = make_map(&tk, k, S, (int64_t)hkv * dh, 128)) != CP_OK) return s;
-  if ((s = make_map(&tv, v, S, (int64_t)hkv * dh, 128)) != CP_OK) return s;
+  if ((s = make_map(&tq, qh, rows, (int64_t)hg * dh, 128)) != CP_OK) return s;
+  if ((s = make_map(&tdo, doh, rows, (int64_t)hg * dh, 128)) != CP_OK) return s;
+  if ((s = make_map(&tk, kh, rows, (int64_t)hkg * dh, 128)) != CP_OK) return s;
+  if ((s = make_map(&tv, vh, rows, (int64_t)hkg * dh, 128)) != CP_OK) return s;
   uint32_t* err = nullptr;
   if ((s = err_word(&err)) != CP_OK) return s;
 
@@ -793,16 +778,19 @@ cp_status cp_ring_attn_bwd(const void* q, const void* k, const void* v, const fl
                      : layout == CP_LAYOUT_STRIPED ? Layout::Striped
                                                    : Layout::Contiguous;
   plan.P = P;
-  plan.hq = hq;
-  plan.hkv = hkv;
+  plan.hq = hg;
+  plan.hkv = hkg;
   plan.causal = mask == CP_MASK_CAUSAL ? 1 : 0;
   plan.striped = lay == Layout::Striped ? 1 : 0;
   plan.n_docs = n_docs;
-  plan.cu_seqlens = cu_seqlens_dev;
+  plan.cu_seqlens = cu_dev;
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)dh);
   plan.scale = scale;
   plan.scale_log2 = scale * 1.4426950408889634f;
-  plan.S = S;
+  plan.S = (int32_t)rows;
+  plan.group_rows = S;
+  plan.out_hq = groups * hg;
+  plan.out_hkv = groups * hkg;
   for (int r = 0; r < P; ++r) {
     const std::vector<Seg> segs = shard_segments(S, P, lay, r);
     plan.nseg[r] = (int)segs.size();
@@ -815,16 +803,16 @@ cp_status cp_ring_attn_bwd(const void* q, const void* k, const void* v, const fl
   plan.dv = dv;
   plan.err = err;
   Docs docs;
-  if (cu_seqlens_host && n_docs > 0) {
-    docs.cu = cu_seqlens_host;
+  if (cu_host && n_docs > 0) {
+    docs.cu = cu_host;
     docs.n = n_docs;
   }
-  cudaError_t e = launch_bwd_prep(dh, o, dout, lse, S, hq, lg, dd, st);
+  cudaError_t e = launch_bwd_prep(dh, o, dout, lse, S, hg, groups, lg, dd, st);
   if (e != cudaSuccess) return cuda_fail(e, "backward prep launch");
   record(g_ev_attn_begin, st);
   for (int side = 0; side < 2; ++side) {
     const bool dq_side = side == 0;
-    const std::vector<uint32_t> items = bwd_items(plan, dq_side, docs);
+    const std::vector<uint32_t> items = bwd_items(plan, groups, dq_side, docs);
     for (size_t base = 0; base < items.size(); base += CP_BWD_MAX_ITEMS) {
       const size_t cnt = std::min(items.size() - base, (size_t)CP_BWD_MAX_ITEMS);
       plan.n_items = (int)cnt;
@@ -835,8 +823,116 @@ cp_status cp_ring_attn_bwd(const void* q, const void* k, const void* v, const fl
     if (dq_side) record(g_ev_merge_end, st);
   }
   record(g_ev_attn_end, st);
+  return CP_OK;
+}
+
+cp_status bwd_check_ptrs(const void* q, const void* k, const void* v, const float* o, const float* lse,
+                         const void* dout, float* dq, float* dk, float* dv) {
+  CP_CHECK_PTR(q);
+  CP_CHECK_PTR(k);
+  CP_CHECK_PTR(v);
+  CP_CHECK_PTR(o);
+  CP_CHECK_PTR(lse);
+  CP_CHECK_PTR(dout);
+  CP_CHECK_PTR(dq);
+  CP_CHECK_PTR(dk);
+  CP_CHECK_PTR(dv);
+  return CP_OK;
+}
+}  // namespace
+
+cp_status cp_ring_attn_bwd(const void* q, const void* k, const void* v, const float* o, const float* lse,
+                           const void* dout, int S, int hq, int hkv, int dh, int P, cp_layout layout, cp_mask mask,
+                           const int32_t* cu_seqlens_host, const int32_t* cu_seqlens_dev, int n_docs,
+                           float softmax_scale, float* dq, float* dk, float* dv, void* workspace, size_t ws_bytes,
+                           void* stream) {
+  cp_status s;
+  if ((s = ring_check(S, hq, hkv, dh, P, layout, mask, CP_BF16, cu_seqlens_host, n_docs)) != CP_OK) return s;
+  if ((s = bwd_check_ptrs(q, k, v, o, lse, dout, dq, dk, dv)) != CP_OK) return s;
+  if (P > CP_BWD_MAX_RANKS) return fail(CP_ERR_UNSUPPORTED, "P = %d (backward supports 1..%d)", P, CP_BWD_MAX_RANKS);
+  if (n_docs > 0 && !cu_seqlens_dev) return fail(CP_ERR_INVALID_ARG, "n_docs > 0 needs cu_seqlens_dev");
+  const size_t need = bwd_workspace(S, hq);
+  if (!workspace || ws_bytes < need)
+    return fail(CP_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws_bytes);
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return fail(CP_ERR_ALIGNMENT, "workspace is not 256-byte aligned");
+  float* lg = static_cast<float*>(workspace);
+  float* dd = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + align256((size_t)S * hq * sizeof(float)));
+  if ((s = run_bwd(q, k, v, dout, dout, o, lse, S, 1, hq, hkv, dh, P, layout, mask, cu_seqlens_host, cu_seqlens_dev,
+                   n_docs, softmax_scale, dq, dk, dv, lg, dd, static_cast<cudaStream_t>(stream))) != CP_OK)
+    return s;
   return ok();
 }
+
+// Workspace of the hybrid backward: head-major bf16 Q, dO [Pu][S][hq/Pu][dh],
+// K, V [Pu][S][hkv/Pu][dh], then D and LSE*log2(e).
+static size_t usp_bwd_workspace(int S, int hq, int hkv, int dh) {
+  return 2 * align256((size_t)S * hq * dh * 2) + 2 * align256((size_t)S * hkv * dh * 2) + bwd_workspace(S, hq);
+}
+
+cp_status cp_usp_attn_bwd_workspace_size(int S, int hq, int hkv, int dh, int Pr, int Pu, cp_layout layout,
+                                         cp_mask mask, const int32_t* cu_seqlens_host, int n_docs, size_t* bytes) {
+  cp_status s;
+  if (!bytes) return fail(CP_ERR_INVALID_ARG, "bytes is NULL");
+  if ((s = usp_check(S, hq, hkv, dh, Pr, Pu, layout, mask, cu_seqlens_host, n_docs)) != CP_OK) return s;
+  *bytes = usp_bwd_workspace(S, hq, hkv, dh);
+  return ok();
+}
+
+cp_status cp_usp_attn_bwd(const void* q, const void* k, const void* v, const float* o, const float* lse,
+                          const void* dout, int S, int hq, int hkv, int dh, int Pr, int Pu, cp_layout layout,
+                          cp_mask mask, const int32_t* cu_seqlens_host, const int32_t* cu_seqlens_dev, int n_docs,
+                          float softmax_scale, float* dq, float* dk, float* dv, void* workspace, size_t ws_bytes,
+                          void* stream) {
+  cp_status s;
+  if ((s = usp_check(S, hq, hkv, dh, Pr, Pu, layout, mask, cu_seqlens_host, n_docs)) != CP_OK) return s;
+  if ((s = bwd_check_ptrs(q, k, v, o, lse, dout, dq, dk, dv)) != CP_OK) return s;
+  if (Pr > CP_BWD_MAX_RANKS) return fail(CP_ERR_UNSUPPORTED, "Pr = %d (backward supports 1..%d)", Pr, CP_BWD_MAX_RANKS);
+  if (Pu > CP_BWD_MAX_GROUPS) return fail(CP_ERR_UNSUPPORTED, "Pu = %d (backward supports 1..%d)", Pu, CP_BWD_MAX_GROUPS);
+  if (n_docs > 0 && !cu_seqlens_dev) return fail(CP_ERR_INVALID_ARG, "n_docs > 0 needs cu_seqlens_dev");
+  const size_t need = usp_bwd_workspace(S, hq, hkv, dh);
+  if (!workspace || ws_bytes < need)
+    return fail(CP_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws_bytes);
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return fail(CP_ERR_ALIGNMENT, "workspace is not 256-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  size_t off = 0;
+  void* qh = ws + off;
+  off += align256((size_t)S * hq * dh * 2);
+  void* doh = ws + off;
+  off += align256((size_t)S * hq * dh * 2);
+  void* kh = ws + off;
+  off += align256((size_t)S * hkv * dh * 2);
+  void* vh = ws + off;
+  off += align256((size_t)S * hkv * dh * 2);
+  float* lg = reinterpret_cast<float*>(ws + off);
+  float* dd = reinterpret_cast<float*>(ws + off + align256((size_t)S * hq * sizeof(float)));
+  const int hg = hq / Pu, hkg = hkv / Pu, n = S / Pu;
+  // Ulysses seq->head of Q, K, V and dO (every group at once); the gradients
+  // and the LSE are read and written in their final layouts by the kernels.
+  cudaError_t e;
+  if ((e = launch_ulysses(q, qh, Pu, n, (size_t)hg * dh * 2, 0, st)) != cudaSuccess ||
+      (e = launch_ulysses(dout, doh, Pu, n, (size_t)hg * dh * 2, 0, st)) != cudaSuccess ||
+      (e = launch_ulysses(k, kh, Pu, n, (size_t)hkg * dh * 2, 0, st)) != cudaSuccess ||
+      (e = launch_ulysses(v, vh, Pu, n, (size_t)hkg * dh * 2, 0, st)) != cudaSuccess)
+    return cuda_fail(e, "usp backward seq->head");
+  if ((s = run_bwd(qh, kh, vh, doh, dout, o, lse, S, Pu, hg, hkg, dh, Pr, layout, mask, cu_seqlens_host,
+                   cu_seqlens_dev, n_docs, softmax_scale, dq, dk, dv, lg, dd, st)) != CP_OK)
+    return s;
+  return ok();
+}
+
+cp_status cp_ulysses_attn_bwd_workspace_size(int S, int hq, int hkv, int dh, int P, size_t* bytes) {
+  return cp_usp_attn_bwd_workspace_size(S, hq, hkv, dh, 1, P, CP_LAYOUT_CONTIGUOUS, CP_MASK_CAUSAL, nullptr, 0, bytes);
+}
+
+cp_status cp_ulysses_attn_bwd(const void* q, const void* k, const void* v, const float* o, const float* lse,
+                              const void* dout, int S, int hq, int hkv, int dh, int P, cp_mask mask,
+                              float softmax_scale, float* dq, float* dk, float* dv, void* workspace, size_t ws_bytes,
+                              void* stream) {
+  return cp_usp_attn_bwd(q, k, v, o, lse, dout, S, hq, hkv, dh, 1, P, CP_LAYOUT_CONTIGUOUS, mask, nullptr, nullptr, 0,
+                         softmax_scale, dq, dk, dv, workspace, ws_bytes, stream);
+}
+
 
 cp_status cp_ring_schedule(int S, int P, cp_layout layout, cp_mask mask, const int32_t* cu_seqlens_host, int n_docs,
                            int32_t* src, int32_t* launched, int32_t* q_rows, int64_t* live_pairs) {

@@ -80,15 +80,17 @@ struct BwdTile {
 };
 
 struct Own {
-  int rank, buf_row0, pos0, valid;
+  int rank, grp, grp_row0, buf_row0, pos0, valid;
 };
 
 __device__ __forceinline__ void decode_own(const cp_bwd_plan& pl, uint32_t item, Own& o) {
-  o.rank = (int)(item >> 24);
-  const int sg = (int)((item >> 23) & 1u);
-  const int tile = (int)(item & 0x7FFFFFu);
+  o.rank = (int)(item >> 26);
+  const int sg = (int)((item >> 25) & 1u);
+  o.grp = (int)((item >> 19) & 63u);
+  const int tile = (int)(item & 0x7FFFFu);
   const cp_seg& s = pl.seg[o.rank][sg];
-  o.buf_row0 = s.buf_row + tile * 128;
+  o.grp_row0 = o.grp * pl.group_rows;
+  o.buf_row0 = o.grp_row0 + s.buf_row + tile * 128;
   o.pos0 = s.pos + tile * 128;
   o.valid = min(128, s.len - tile * 128);
 }
@@ -103,12 +105,13 @@ struct KvTile {
 // Every role of the CTA runs its own copy and sees the same sequence.
 struct DqIter {
   const cp_bwd_plan* pl;
-  int r, t, sg, tl;
+  int r, t, sg, tl, row0;
   int vis_lo, vis_hi, full_lo, full_hi;
 
   __device__ void init(const cp_bwd_plan& p, const Own& own) {
     pl = &p;
     r = own.rank;
+    row0 = own.grp_row0;
     t = sg = tl = 0;
     const int qa = own.pos0, qb = own.pos0 + own.valid - 1;
     const bool docs = p.n_docs > 0;
@@ -144,7 +147,7 @@ struct DqIter {
       const int valid = min(128, s.len - off);
       const int kb = ka + valid - 1;
       if (kb >= vis_lo && ka <= vis_hi) {
-        out.buf_row = s.buf_row + off;
+        out.buf_row = row0 + s.buf_row + off;
         out.pos = ka;
         out.valid = valid;
         out.full = valid == 128 && ka >= full_lo && kb <= full_hi;
@@ -431,7 +434,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (ok) {
       // warpgroup hh writes dQ columns [hh DH/2, (hh + 1) DH/2)
       tc_fence_after();
-      float* dst = plan.dq + ((size_t)(own.buf_row0 + row) * plan.hq + h) * DH + hh * (DH / 2);
+      const size_t orow = (size_t)(own.buf_row0 - own.grp_row0 + row);
+      float* dst = plan.dq + (orow * plan.out_hq + own.grp * plan.hq + h) * DH + hh * (DH / 2);
 #pragma unroll 1
       for (int ch = 0; ch < DH / 64; ++ch) {
         uint32_t o[32];
@@ -474,7 +478,7 @@ struct QTile {
 // step t, then their tiles.
 struct KvIter {
   const cp_bwd_plan* pl;
-  int j, hk, g, t, sg, tl;
+  int j, hk, g, t, sg, tl, row0;
   int ka0, kb0;                    // own positions without the striped shift
   int lo0, hi0, flo0, fhi0;        // windows of admitted query positions
 
@@ -482,6 +486,7 @@ struct KvIter {
     pl = &p;
     j = own.rank;
     hk = kv_head;
+    row0 = own.grp_row0;
     g = t = sg = tl = 0;
     ka0 = own.pos0;
     kb0 = own.pos0 + own.valid - 1;
@@ -526,7 +531,7 @@ struct KvIter {
       const int valid = min(128, s.len - off);
       const int qb = qa + valid - 1;
       if (qb >= lo0 + shift && qa <= hi0) {
-        out.buf_row = s.buf_row + off;
+        out.buf_row = row0 + s.buf_row + off;
         out.pos = qa;
         out.valid = valid;
         out.h = hk * group + g;
@@ -864,7 +869,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (ok) {
       // warpgroup 0 writes dV, warpgroup 1 writes dK * scale
       tc_fence_after();
-      const size_t orow = (size_t)(own.buf_row0 + row) * plan.hkv + hk;
+      const size_t orow = (size_t)(own.buf_row0 - own.grp_row0 + row) * plan.out_hkv + own.grp * plan.hkv + hk;
       float* dst = (hh == 0 ? plan.dv : plan.dk) + orow * DH;
       const uint32_t col = hh == 0 ? C::kColDV : C::kColDK;
       const float f = hh == 0 ? 1.f : plan.scale;
@@ -901,17 +906,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
 // ------------------------------------------------------------------ prep
 // D = rowsum(dO * O) and LSE * log2(e) per (row, head), one warp per pair.
+// The outputs are [hg][groups * G] (plan rows: group g's rows start at g G);
+// O, dO are read in their final [G][groups * hg][dh] layout and LSE in its
+// final [groups * hg][G] layout, group g holding heads [g hg, (g + 1) hg).
 template <int DH>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const float* __restrict__ o, const uint16_t* __restrict__ dout,
-                                                       const float* __restrict__ lse, int S, int hq,
-                                                       float* __restrict__ lg, float* __restrict__ dd) {
+                                                       const float* __restrict__ lse, int rows, int G, int hg,
+                                                       int groups, float* __restrict__ lg, float* __restrict__ dd) {
   constexpr int E = DH / 32;
   const long long item = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (item >= (long long)S * hq) return;
+  if (item >= (long long)rows * hg) return;
   const int lane = threadIdx.x & 31;
-  const int row = (int)(item / hq);
-  const int h = (int)(item - (long long)row * hq);
-  const size_t base = ((size_t)row * hq + h) * DH + (size_t)lane * E;
+  const int row = (int)(item / hg);
+  const int h = (int)(item - (long long)row * hg);
+  const int g = row / G, x = row - g * G;
+  const int hq = groups * hg;
+  const size_t base = ((size_t)x * hq + g * hg + h) * DH + (size_t)lane * E;
   float acc = 0.f;
   if constexpr (E == 4) {
     const float4 a = __ldcs(reinterpret_cast<const float4*>(o + base));
@@ -926,8 +936,8 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const float* __restrict__
 #pragma unroll
   for (int m = 16; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
   if (lane == 0) {
-    const size_t v = (size_t)h * S + row;
-    const float l = lse[v];
+    const size_t v = (size_t)h * rows + row;
+    const float l = lse[((size_t)g * hg + h) * G + x];
     dd[v] = acc;
     lg[v] = l == -CUDART_INF_F ? 0.f : l * kLog2e;
   }
@@ -958,15 +968,17 @@ cudaError_t launch_bwd_dh(const CUtensorMap& tq, const CUtensorMap& tdo, const C
 
 }  // namespace
 
-cudaError_t launch_bwd_prep(int dh, const float* o, const void* dout, const float* lse, int S, int hq, float* lg,
-                            float* dd, cudaStream_t st) {
-  const long long items = (long long)S * hq;
+// rows = groups * G plan rows, hg heads per group.
+cudaError_t launch_bwd_prep(int dh, const float* o, const void* dout, const float* lse, int G, int hg, int groups,
+                            float* lg, float* dd, cudaStream_t st) {
+  const int rows = G * groups;
+  const long long items = (long long)rows * hg;
   if (items <= 0) return cudaSuccess;
   const unsigned grid = (unsigned)((items + 7) / 8);
   if (dh == 128)
-    bwd_prep_kernel<128><<<grid, 256, 0, st>>>(o, static_cast<const uint16_t*>(dout), lse, S, hq, lg, dd);
+    bwd_prep_kernel<128><<<grid, 256, 0, st>>>(o, static_cast<const uint16_t*>(dout), lse, rows, G, hg, groups, lg, dd);
   else
-    bwd_prep_kernel<64><<<grid, 256, 0, st>>>(o, static_cast<const uint16_t*>(dout), lse, S, hq, lg, dd);
+    bwd_prep_kernel<64><<<grid, 256, 0, st>>>(o, static_cast<const uint16_t*>(dout), lse, rows, G, hg, groups, lg, dd);
   launch_counter()++;
   return cudaGetLastError();
 }

@@ -93,9 +93,13 @@ struct cp_merge_plan {
 // tile of shard j and the partners are the ranks (j + t) mod P that hold it at
 // step t (and every query head of its group).
 //
-// item: (rank << 24) | (segment << 23) | tile, tile = 128-row tile index
-// inside the segment.  Striped layouts carry local row indices as positions;
-// a key of shard j seen from rank r then sits one position later when j > r.
+// item: (rank << 26) | (segment << 25) | (group << 19) | tile, tile =
+// 128-row tile index inside the segment.  A group is a block of heads whose
+// rows start at group * group_rows in the Q/K/V/dO buffers (the head-major
+// layout of the Ulysses transpose; one group for the plain ring).  Striped
+// layouts carry local row indices as positions; a key of shard j seen from
+// rank r then sits one position later when j > r.
+#define CP_BWD_MAX_GROUPS 64
 struct cp_bwd_plan {
   int32_t P;
   int32_t hq, hkv;
@@ -106,13 +110,15 @@ struct cp_bwd_plan {
   float scale_log2;             // softmax_scale * log2(e)
   float scale;
   int32_t S;                    // rows of every buffer (row pitch of lg, dd)
+  int32_t group_rows;           // rows per head group in the buffers
+  int32_t out_hq, out_hkv;      // heads per row of dq and of dk, dv (all groups)
   int32_t nseg[CP_BWD_MAX_RANKS];
   cp_seg seg[CP_BWD_MAX_RANKS][2];
   const float* lg;              // [hq][S]: LSE * log2(e) (0 where LSE = -inf)
   const float* dd;              // [hq][S]: rowsum(dO * O)
-  float* dq;                    // [S][hq][dh]
-  float* dk;                    // [S][hkv][dh]
-  float* dv;                    // [S][hkv][dh]
+  float* dq;                    // [group_rows][out_hq][dh]: group g holds heads [g hq, (g + 1) hq)
+  float* dk;                    // [group_rows][out_hkv][dh]
+  float* dv;                    // [group_rows][out_hkv][dh]
   uint32_t* err;
   int32_t n_items;
   uint32_t items[CP_BWD_MAX_ITEMS];

@@ -290,6 +290,44 @@ cp_status cp_ring_attn_bwd(const void* q, const void* k, const void* v, const fl
                            void* stream);
 
 /*
+ * cp_usp_attn_bwd_workspace_size / cp_usp_attn_bwd -- gradients of
+ * cp_usp_attn_fwd (the Ulysses-inside / Ring-across hybrid) for an upstream
+ * gradient dO, with the same rank grid, layouts and support as the forward.
+ * Inputs (device, in the forward's storage order): q [S][hq][dh], k, v
+ * [S][hkv][dh], dout [S][hq][dh] bf16; o [S][hq][dh] fp32 and lse [hq][S]
+ * fp32 from the forward.  Outputs (fp32, fully overwritten, same order): dq
+ * [S][hq][dh], dk and dv [S][hkv][dh].
+ * Steps: Ulysses seq->head transpose of Q, K, V and dO over Pu; for every
+ * head block, the ring backward of cp_ring_attn_bwd over the Pr groups (one
+ * dQ launch and one dK/dV launch cover all head blocks); the kernels read O
+ * and LSE and write dq, dk, dv directly in the final layouts, which is the
+ * head->seq transpose of the gradients.
+ * Workspace: caller-owned, 256-byte aligned, size from
+ * cp_usp_attn_bwd_workspace_size (head-major Q, dO, K, V and two fp32
+ * [hq][S] vectors).  Errors as cp_usp_attn_fwd; nothing is launched on error.
+ */
+cp_status cp_usp_attn_bwd_workspace_size(int S, int hq, int hkv, int dh, int Pr, int Pu, cp_layout layout,
+                                         cp_mask mask, const int32_t* cu_seqlens_host, int n_docs, size_t* bytes);
+cp_status cp_usp_attn_bwd(const void* q, const void* k, const void* v, const float* o, const float* lse,
+                          const void* dout, int S, int hq, int hkv, int dh, int Pr, int Pu, cp_layout layout,
+                          cp_mask mask, const int32_t* cu_seqlens_host, const int32_t* cu_seqlens_dev, int n_docs,
+                          float softmax_scale, float* dq, float* dk, float* dv, void* workspace, size_t ws_bytes,
+                          void* stream);
+
+/*
+ * cp_ulysses_attn_bwd_workspace_size / cp_ulysses_attn_bwd -- gradients of
+ * cp_ulysses_attn_fwd: the hybrid backward with Pr = 1 and Pu = P (every
+ * rank's head group attends over the whole sequence).  Inputs and outputs
+ * in the forward's natural sequence order, dtypes as cp_usp_attn_bwd.
+ * Supported: P | hkv, P | S, dh in {64, 128}.
+ */
+cp_status cp_ulysses_attn_bwd_workspace_size(int S, int hq, int hkv, int dh, int P, size_t* bytes);
+cp_status cp_ulysses_attn_bwd(const void* q, const void* k, const void* v, const float* o, const float* lse,
+                              const void* dout, int S, int hq, int hkv, int dh, int P, cp_mask mask,
+                              float softmax_scale, float* dq, float* dk, float* dv, void* workspace, size_t ws_bytes,
+                              void* stream);
+
+/*
  * Host-only inspection of the ring-step schedule (no GPU needed).  For every
  * rank r and step t (index r*P + t):
  *   src[r*P+t]        the key/value shard j = (r - t) mod P held at that step

@@ -1,5 +1,5 @@
-"""GPU parity of the ring backward (prep, dQ kernel, dK/dV kernel) against
-the fp64 oracle's gradient of the exact attention.
+"""GPU parity of the backward (prep, dQ kernel, dK/dV kernel; ring, Ulysses
+and the hybrid) against the fp64 oracle's gradient of the exact attention.
 
 Tolerance, derived from the arithmetic: the kernels round P and dS to bf16
 (unit roundoff u = 2^-8) before the tensor-core products and accumulate in
@@ -149,3 +149,55 @@ def test_bwd_full_size_32k():
     sum_dv = f64(dv.sum(dim=0))
     want_dv = f64(do.float().sum(dim=0))
     assert np.max(np.abs(sum_dv - want_dv)) <= 2e-2 * np.max(np.abs(want_dv)), "sum over keys of dV != sum of dO"
+
+
+# ----------------------------------------------------------- Ulysses and the hybrid
+def usp_bwd_case(S, hq, hkv, dh, Pr, Pu, layout, causal=True, cu=None):
+    q, k, v = synth.qkv(S, hq, hkv, dh)
+    do = synth.normal((S, hq, dh), synth.SEED_DO, 0.5)
+    order = storage_order(S, Pr, layout)
+    idx = torch.from_numpy(order)
+    qs, ks, vs, dos = (t[idx].contiguous().cuda() for t in (q, k, v, do))
+    o, lse = api.usp_attn_fwd(qs, ks, vs, Pr, Pu, layout, causal, cu)
+    dq, dk, dv = api.usp_attn_bwd(qs, ks, vs, o, lse, dos, Pr, Pu, layout, causal, cu)
+    torch.cuda.synchronize()
+    assert api.device_error() == 0
+    wq, wk, wv = ref.attention_bwd(f64(q), f64(k), f64(v), f64(do), causal=causal, cu_seqlens=cu)
+    what = f"usp S={S} Pr={Pr} Pu={Pu} {layout}"
+    check_grad(dq, wq[order], "dQ " + what)
+    check_grad(dk, wk[order], "dK " + what)
+    check_grad(dv, wv[order], "dV " + what)
+
+
+@pytest.mark.parametrize("layout", ["contiguous", "zigzag", "striped"])
+@pytest.mark.parametrize("Pr,Pu", [(2, 2), (1, 4), (4, 2)])
+def test_usp_bwd(layout, Pr, Pu):
+    usp_bwd_case(1024, 8, 4, 128, Pr, Pu, layout)
+
+
+def test_usp_bwd_documents_noncausal_dh64():
+    S = 2048
+    lens = synth.doc_lengths(S, 64, 700, seed=6)
+    usp_bwd_case(S, 4, 2, 64, 2, 2, "zigzag", causal=False, cu=synth.cu_seqlens_from_lengths(lens).tolist())
+
+
+def test_usp_bwd_many_items():
+    # 8 zigzag ring ranks x 4 head blocks: 256 own tiles of four head blocks
+    # interleaved in one launch per kernel
+    usp_bwd_case(8192, 8, 4, 64, 8, 4, "zigzag")
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_ulysses_bwd(causal):
+    S, hq, hkv, dh, P = 1024, 8, 4, 128, 4
+    q, k, v = synth.qkv(S, hq, hkv, dh)
+    do = synth.normal((S, hq, dh), synth.SEED_DO, 0.5)
+    qd, kd, vd, dod = (t.cuda() for t in (q, k, v, do))
+    o, lse = api.ulysses_attn_fwd(qd, kd, vd, P, causal=causal)
+    dq, dk, dv = api.ulysses_attn_bwd(qd, kd, vd, o, lse, dod, P, causal=causal)
+    torch.cuda.synchronize()
+    assert api.device_error() == 0
+    wq, wk, wv = ref.attention_bwd(f64(q), f64(k), f64(v), f64(do), causal=causal)
+    check_grad(dq, wq, "ulysses dQ")
+    check_grad(dk, wk, "ulysses dK")
+    check_grad(dv, wv, "ulysses dV")

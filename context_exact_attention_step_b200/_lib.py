@@ -27,6 +27,7 @@ EXPORTS = [
     "cp_ring_attn_fwd_noalloc", "cp_selftest_wait_timeout", "cp_striped_reorder",
     "cp_usp_attn_workspace_size", "cp_usp_attn_fwd", "cp_ring_attn_bwd_workspace_size", "cp_ring_attn_bwd",
     "cp_usp_attn_bwd_workspace_size", "cp_usp_attn_bwd", "cp_ulysses_attn_bwd_workspace_size", "cp_ulysses_attn_bwd",
+    "cp_head_block_split",
 ]
 
 
@@ -77,6 +78,8 @@ def lib():
     L.cp_ulysses_permute.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, vp]
     L.cp_striped_reorder.restype = i32
     L.cp_striped_reorder.argtypes = [vp, vp, i32, i32, i32, i32, i32, vp]
+    L.cp_head_block_split.restype = i32
+    L.cp_head_block_split.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, vp]
     L.cp_zigzag_reorder.restype = i32
     L.cp_zigzag_reorder.argtypes = [vp, vp, i32, i32, i32, i32, i32, vp]
     L.cp_ulysses_attn_workspace_size.restype = i32

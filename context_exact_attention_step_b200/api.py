@@ -192,6 +192,24 @@ def ulysses_permute(x, P, direction="seq_to_head", out=None, stream=None):
     return out
 
 
+def head_block_split(x, P, inverse=False, out=None, stream=None):
+    """inverse=False: x [n, h, dh] -> [P, n, h/P, dh] (block r for rank r);
+    inverse=True: x [P, n, h/P, dh] -> [n, h, dh].  Bit-exact copy."""
+    _need_cuda("x", x)
+    if not inverse:
+        n, h, dh = x.shape
+        shape = (P, n, h // P, dh)
+    else:
+        p_, n, hg, dh = x.shape
+        h = hg * P
+        shape = (n, h, dh)
+    if out is None:
+        out = torch.empty(shape, device=x.device, dtype=x.dtype)
+    check(lib().cp_head_block_split(_vp(x), _vp(out), n, h, dh, P, x.element_size(), 1 if inverse else 0,
+                                    _stream(stream)))
+    return out
+
+
 def zigzag_reorder(x, P, inverse=False, seq_dim=0, out=None, stream=None):
     """Natural <-> rank-major zigzag order along ``seq_dim`` (0 for [S, ...]
     tensors, 1 for [h, S] LSE tensors)."""

@@ -29,6 +29,8 @@ cudaError_t launch_ulysses(const void* in, void* out, int P, int n, size_t chunk
 cudaError_t launch_zigzag(const void* in, void* out, int P, int batch, size_t chunk_bytes, int inverse,
                           cudaStream_t st);
 cudaError_t launch_f32_to_bf16(const float* in, void* out, size_t n, cudaStream_t st);
+cudaError_t launch_head_blocks(const void* in, void* out, int P, int n, size_t chunk_bytes, int inverse,
+                               cudaStream_t st);
 cudaError_t launch_striped(const void* in, void* out, int P, int S, int batch, size_t row_bytes, int inverse,
                            cudaStream_t st);
 cudaError_t launch_bwd_prep(int dh, const float* o, const void* dout, const float* lse, int G, int hg, int groups,
@@ -495,6 +497,22 @@ cp_status cp_zigzag_reorder(const void* in, void* out, int P, int S, int batch, 
   const size_t chunk = (size_t)(S / (2 * P)) * row_bytes;
   cudaError_t e = launch_zigzag(in, out, P, batch, chunk, inverse ? 1 : 0, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "zigzag reorder launch");
+  return ok();
+}
+
+cp_status cp_head_block_split(const void* in, void* out, int n, int h, int dh, int P, int elem_bytes, int inverse,
+                              void* stream) {
+  if (!in || !out) return fail(CP_ERR_INVALID_ARG, "in/out is NULL");
+  if (P < 1 || n <= 0 || h <= 0 || dh <= 0) return fail(CP_ERR_INVALID_ARG, "sizes must be positive");
+  if (elem_bytes != 1 && elem_bytes != 2 && elem_bytes != 4 && elem_bytes != 8)
+    return fail(CP_ERR_INVALID_ARG, "elem_bytes = %d", elem_bytes);
+  if (h % P != 0) return fail(CP_ERR_UNSUPPORTED, "heads (%d) must be a multiple of P (%d)", h, P);
+  const size_t bytes = (size_t)n * h * dh * elem_bytes;
+  const uint8_t *a = static_cast<const uint8_t*>(in), *b = static_cast<const uint8_t*>(out);
+  if (a < b + bytes && b < a + bytes) return fail(CP_ERR_INVALID_ARG, "in and out overlap");
+  cudaError_t e = launch_head_blocks(in, out, P, n, (size_t)(h / P) * dh * elem_bytes, inverse ? 1 : 0,
+                                     static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "head-block split launch");
   return ok();
 }
 

@@ -10,6 +10,9 @@
 //    timeline: Striped / zigzag load-balancing reorder), and its inverse.
 //  * Striped reorder: token t on rank t mod P (same timeline, Striped
 //    Attention), and its inverse.
+//  * Head-block split of one rank's rows for the Ulysses all-to-all:
+//    out[r][s][h'] = in[s][r*H/P + h'] (the send buffer whose block r goes
+//    to rank r), and its inverse after the exchange.
 //  * fp32 -> bf16 round-to-nearest-even conversion of input tensors.
 //
 // Both layout changes move whole runs of >= 256 contiguous bytes (one head
@@ -123,6 +126,36 @@ __global__ void __launch_bounds__(256) striped_kernel(const U* __restrict__ in, 
       irow = r * n + a;
     }
     st_stream(out + base + (size_t)orow * upr + c, ld_stream(in + base + (size_t)irow * upr + c));
+  }
+}
+
+// Head blocks: in [n][P][cu] <-> out [P][n][cu] (cu units per head block).
+template <typename U, int ILP>
+__global__ void __launch_bounds__(256) head_block_kernel(const U* __restrict__ in, U* __restrict__ out, int P, int n,
+                                                         uint32_t cu, int inverse) {
+  const int r = blockIdx.y;
+  const uint32_t total = (uint32_t)n * cu;
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  for (size_t u0 = (size_t)blockIdx.x * blockDim.x + threadIdx.x; u0 < total; u0 += stride * ILP) {
+    U v[ILP];
+    size_t dst[ILP];
+#pragma unroll
+    for (int i = 0; i < ILP; ++i) {
+      const size_t u = u0 + i * stride;
+      if (u < total) {
+        const uint32_t s = (uint32_t)u / cu;
+        const uint32_t c = (uint32_t)u - s * cu;
+        const size_t seq_major = ((size_t)s * P + r) * cu + c;
+        const size_t block_major = (size_t)r * total + u;
+        dst[i] = inverse ? seq_major : block_major;
+        v[i] = ld_stream(in + (inverse ? block_major : seq_major));
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < ILP; ++i) {
+      const size_t u = u0 + i * stride;
+      if (u < total) st_stream(out + dst[i], v[i]);
+    }
   }
 }
 
@@ -244,6 +277,29 @@ cudaError_t launch_striped(const void* in, void* out, int P, int S, int batch, s
     case 4: return striped_t<uint32_t>(in, out, P, n, batch, row_bytes, inverse, st);
     case 2: return striped_t<uint16_t>(in, out, P, n, batch, row_bytes, inverse, st);
     default: return striped_t<uint8_t>(in, out, P, n, batch, row_bytes, inverse, st);
+  }
+}
+
+template <typename U>
+static cudaError_t head_block_t(const void* in, void* out, int P, int n, size_t chunk_bytes, int inverse,
+                                cudaStream_t st) {
+  constexpr int ILP = 4;
+  const uint32_t cu = (uint32_t)(chunk_bytes / sizeof(U));
+  dim3 grid(grid_x((size_t)n * cu, ILP, (unsigned)P), (unsigned)P);
+  head_block_kernel<U, ILP><<<grid, 256, 0, st>>>(static_cast<const U*>(in), static_cast<U*>(out), P, n, cu,
+                                                   inverse);
+  launch_counter()++;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_head_blocks(const void* in, void* out, int P, int n, size_t chunk_bytes, int inverse,
+                               cudaStream_t st) {
+  switch (unit_bytes(chunk_bytes, in, out)) {
+    case 16: return head_block_t<uint4>(in, out, P, n, chunk_bytes, inverse, st);
+    case 8: return head_block_t<uint2>(in, out, P, n, chunk_bytes, inverse, st);
+    case 4: return head_block_t<uint32_t>(in, out, P, n, chunk_bytes, inverse, st);
+    case 2: return head_block_t<uint16_t>(in, out, P, n, chunk_bytes, inverse, st);
+    default: return head_block_t<uint8_t>(in, out, P, n, chunk_bytes, inverse, st);
   }
 }
 

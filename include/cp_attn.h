@@ -193,6 +193,18 @@ cp_status cp_zigzag_reorder(const void* in, void* out, int P, int S, int batch, 
                             void* stream);
 
 /*
+ * cp_head_block_split -- the local half of the Ulysses all-to-all when every
+ * rank is its own GPU ("序列並行" concept page (compassingai), 技術原理 §三;
+ * "Context Parallelism" write-up (pwwt.cn) §2.3): one rank's rows in [n][h][dh]
+ * are regrouped by head block, out [P][n][h/P][dh], out[r][s][h'] =
+ * in[s][r*h/P + h'], so that block r can be sent to rank r; inverse = 1 undoes
+ * it after the exchange.  Bit-exact copy of elem_bytes-sized elements.
+ * Supported: P | h; in and out must not overlap.
+ */
+cp_status cp_head_block_split(const void* in, void* out, int n, int h, int dh, int P, int elem_bytes, int inverse,
+                              void* stream);
+
+/*
  * cp_striped_reorder -- natural token order <-> rank-major striped order
  * (token t on rank t mod P, rank r's rows in position order: row r*S/P + a
  * holds position a*P + r).  in/out are [batch][S][row_bytes] byte arrays as

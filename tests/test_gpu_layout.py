@@ -88,3 +88,14 @@ def test_zigzag_lse_rows():
     y = api.zigzag_reorder(lse, P, seq_dim=1)
     assert np.array_equal(bits(y), ref.zigzag_reorder(bits(lse), P, axis=1))
     assert torch.equal(api.zigzag_reorder(y, P, inverse=True, seq_dim=1), lse)
+
+
+@pytest.mark.parametrize("P,elem", [(2, torch.bfloat16), (4, torch.float32), (8, torch.bfloat16)])
+def test_head_block_split_bit_exact(P, elem):
+    n, h, dh = 300, 16, 64
+    x = synth.normal((n, h, dh), 9, 1.0, dtype=torch.float32).to(elem)
+    y = api.head_block_split(x.cuda(), P)
+    want = x.reshape(n, P, h // P, dh).permute(1, 0, 2, 3).contiguous()
+    assert torch.equal(y.cpu(), want)
+    back = api.head_block_split(y, P, inverse=True)
+    assert torch.equal(back.cpu(), x)

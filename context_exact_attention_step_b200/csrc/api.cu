@@ -230,11 +230,22 @@ struct MergeTaskIn {
 
 // o_heads: heads per output row of O (h unless tasks scatter head blocks
 // into a wider output through head_off).
-cp_status run_merge(const std::vector<MergeTaskIn>& tasks, int h, int dh, float* o_out, float* lse_out,
+cp_status run_merge(const std::vector<MergeTaskIn>& tasks_in, int h, int dh, float* o_out, float* lse_out,
                     int lse_out_ld, void* o_bf16, cudaStream_t st, int o_heads = 0) {
   static cp_merge_plan plan;
   static std::mutex mu;
   std::lock_guard<std::mutex> lk(mu);
+  // Tasks with more partials per row first: CTAs start in task order, so the
+  // long ones do not form the tail of the launch.
+  std::vector<const MergeTaskIn*> order;
+  order.reserve(tasks_in.size());
+  for (const MergeTaskIn& t : tasks_in) order.push_back(&t);
+  std::stable_sort(order.begin(), order.end(), [](const MergeTaskIn* a, const MergeTaskIn* b) {
+    return (int64_t)a->in.size() * a->rows > (int64_t)b->in.size() * b->rows;
+  });
+  std::vector<MergeTaskIn> tasks;
+  tasks.reserve(order.size());
+  for (const MergeTaskIn* t : order) tasks.push_back(*t);
   size_t i = 0;
   while (i < tasks.size()) {
     memset(&plan, 0, sizeof(plan));

@@ -105,6 +105,11 @@ def test_ring_over_ranks(layout, world):
     _run("ring", world, dict(S=64, hq=4, hkv=2, dh=8, layout=layout, causal=True))
 
 
+def test_ring_over_three_ranks():
+    # an odd ring: every rank's shard visits the others in the same order
+    _run("ring", 3, dict(S=48, hq=2, hkv=1, dh=8, layout="zigzag", causal=True))
+
+
 def test_ring_over_ranks_noncausal_documents():
     _run("ring", 4, dict(S=64, hq=2, hkv=2, dh=8, layout="zigzag", causal=False, cu=[0, 5, 6, 40, 64]))
     _run("ring", 2, dict(S=64, hq=2, hkv=2, dh=8, layout="contiguous", causal=True, cu=[0, 5, 6, 40, 64]))

@@ -201,3 +201,19 @@ def test_ulysses_bwd(causal):
     check_grad(dq, wq, "ulysses dQ")
     check_grad(dk, wk, "ulysses dK")
     check_grad(dv, wv, "ulysses dV")
+
+
+def test_bwd_sixteen_ranks():
+    # the backward's rank limit: 16 zigzag shards of 128 rows
+    bwd_case(4096, 2, 2, 64, 16, "zigzag")
+
+
+def test_bwd_ragged_shards():
+    # 3 ranks of 500 rows: every shard ends in a 116-row tile
+    bwd_case(1500, 2, 2, 128, 3, "contiguous")
+
+
+def test_bwd_gqa_documents():
+    S = 2048
+    lens = synth.doc_lengths(S, 50, 600, seed=10)
+    bwd_case(S, 8, 2, 64, 4, "zigzag", cu=synth.cu_seqlens_from_lengths(lens).tolist())

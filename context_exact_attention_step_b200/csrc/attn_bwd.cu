@@ -163,8 +163,10 @@ struct DqCfg {
   using T = BwdTile<DH>;
   static constexpr int kStages = DH == 128 ? 4 : 8;
   static constexpr int kSmemBytes = 1024 + 2 * T::kTileBytes + kStages * T::kTileBytes + 256;
-  // TMEM: S | dP (two buffers; dS is written over its dP) | dQ
-  static constexpr uint32_t kColS = 0, kColD0 = 128, kColD1 = 256, kColQ = 384;
+  // TMEM: S | dP (dS is written over it) | dQ | Q and dO as the A operands of
+  // S = Q K^T and dP = dO V^T, copied in once so that these MMAs read only
+  // K and V from shared memory
+  static constexpr uint32_t kColS = 0, kColD = 128, kColQ = 256, kColQA = 256 + DH, kColDOA = kColQA + DH / 2;
 };
 
 template <int DH>
@@ -181,7 +183,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint8_t* sKV = smem + 2 * T::kTileBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + C::kStages * T::kTileBytes);
   const int B_QD = 0, B_FULL = 1, B_EMPTY = 1 + C::kStages, B_S = 1 + 2 * C::kStages, B_DP = B_S + 1,
-            B_SC = B_DP + 1, B_DS = B_SC + 1, B_ACC = B_DS + 1, B_DRAIN = B_ACC + 1, B_COUNT = B_DRAIN + 1;
+            B_SC = B_DP + 1, B_DS = B_SC + 1, B_ACC = B_DS + 1, B_A = B_ACC + 1, B_DRAIN = B_A + 1,
+            B_COUNT = B_DRAIN + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + B_COUNT);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   auto bar = [&](int i) { return smem_addr(bars + i); };
@@ -200,6 +203,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(bar(B_SC), 8);  // one arrive per element-wise warp
     mbar_init(bar(B_DS), 8);
     mbar_init(bar(B_ACC), 1);
+    mbar_init(bar(B_A), 8);   // Q and dO copied into TMEM by the element-wise warps
     mbar_init(bar(B_DRAIN), 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -223,7 +227,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int hk = h / (plan.hq / plan.hkv);
   Own own;
   decode_own(plan, plan.items[blockIdx.x / plan.hq], own);
-  auto col_d = [](int j) { return (j & 1) ? C::kColD1 : C::kColD0; };
+  auto col_d = [](int) { return C::kColD; };
 
   // Registers: launched at 168 per thread (384 threads); inside its own
   // branch the control warpgroup (warps 0-3) drops to 64 and the two
@@ -264,15 +268,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     constexpr uint32_t idesc_ss = idesc_bf16_f32(128, 128, false);
     constexpr uint32_t idesc_dq = idesc_bf16_f32(128, DH, true);
-    const uint32_t sq = smem_addr(sQ), sdo = smem_addr(sDO), skv = smem_addr(sKV);
-    // D[col] = A B^T over dh, both operands K-major 128-row tiles
-    auto issue_ss = [&](uint32_t dcol, uint32_t a_base, uint32_t b_base) {
+    const uint32_t skv = smem_addr(sKV);
+    const uint32_t sq = C::kColQA, sdo = C::kColDOA;  // A operands, in TMEM
+    // D[col] = A B^T over dh: A (Q or dO, bf16 in TMEM at column acol, 8
+    // columns per K-step of 16) times a K-major 128-row key/value tile
+    auto issue_ss = [&](uint32_t dcol, uint32_t acol, uint32_t b_base) {
 #pragma unroll
       for (int kk = 0; kk < DH / 16; ++kk) {
         const uint32_t box = kk >> 2, koff = (kk & 3) * 32;
-        const uint64_t a = sdesc_sw128(a_base + box * T::kBoxBytes + koff, 16, 1024);
         const uint64_t b = sdesc_sw128(b_base + box * T::kBoxBytes + koff, 16, 1024);
-        tc_mma_ss_elect(tmem + dcol, a, b, idesc_ss, kk > 0 ? 1u : 0u);
+        tc_mma_ts_elect(tmem + dcol, tmem + acol + kk * 8, b, idesc_ss, kk > 0 ? 1u : 0u);
       }
     };
     // dQ += dS K: A = dS (bf16 in TMEM, 128 keys as 8 K-steps of 16; keys
@@ -291,7 +296,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     auto vph = [&](int j) { return (uint32_t)(((2 * j + 1) / C::kStages) & 1); };
     auto slot_addr = [&](int s) { return skv + (uint32_t)s * T::kTileBytes; };
 
-    bool ok = mbar_wait_warp(bar(B_QD), 0, abort_flag, err, kWaitNs);
+    bool ok = mbar_wait_warp(bar(B_A), 0, abort_flag, err, kWaitNs);
     DqIter it;
     it.init(plan, own);
     KvTile cur, nxt;
@@ -367,12 +372,40 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint64_t nd2 = f2_pack(-dd, -dd);
     const int c0 = hh * 64;
     const uint32_t ds_off = hh ? 64u : 0u;
+    bool ok = true;
+    {
+      // copy this row of Q (warpgroup 0) or dO (warpgroup 1) from its
+      // 128-byte-swizzled shared tile (16-byte chunk c of row r stored at
+      // chunk c ^ (r & 7)) into TMEM, two bf16 per column
+      ok = mbar_wait(bar(B_QD), 0, abort_flag, err, kWaitNs);
+      ok = __all_sync(0xffffffffu, ok);
+      if (ok) {
+        const uint8_t* src = (hh == 0 ? sQ : sDO) + row * 128;
+        const uint32_t dst = tmem + lane_base + (hh == 0 ? C::kColQA : C::kColDOA);
+#pragma unroll
+        for (int b = 0; b < T::kBoxes; ++b) {
+          uint32_t w[32];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint4 v = *reinterpret_cast<const uint4*>(src + b * T::kBoxBytes + ((c ^ (row & 7)) << 4));
+            w[4 * c + 0] = v.x;
+            w[4 * c + 1] = v.y;
+            w[4 * c + 2] = v.z;
+            w[4 * c + 3] = v.w;
+          }
+          tmem_st32(dst + b * 32, w);
+        }
+        tc_wait_st();
+        tc_fence_before();
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_A));
+    }
     DqIter it;
     it.init(plan, own);
     KvTile kt;
     int j = 0;
-    bool ok = true;
-    while (it.next(kt)) {
+    while (ok && it.next(kt)) {
       ok = mbar_wait(bar(B_S), j & 1u, abort_flag, err, kWaitNs);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;

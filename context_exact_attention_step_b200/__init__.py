@@ -7,6 +7,8 @@ The compute lives in ``libcp_attn.so`` (C ABI in ``include/cp_attn.h``);
 ``api`` is a thin PyTorch binding over it.
 """
 from .api import (  # noqa: F401
+    attn_bwd_prep,
+    block_attn_bwd,
     block_attn_fwd,
     count_live_pairs,
     device_error,

@@ -15,6 +15,8 @@ CP_MASK_NONE, CP_MASK_CAUSAL = 0, 1
 CP_LAYOUT_CONTIGUOUS, CP_LAYOUT_ZIGZAG, CP_LAYOUT_STRIPED = 0, 1, 2
 CP_SEQ_TO_HEAD, CP_HEAD_TO_SEQ = 0, 1
 CP_MAX_CHUNKS = 4
+CP_BWD_DQ, CP_BWD_DKDV = 1, 2
+CP_BWD_MAX_CHUNKS = 2
 
 STATUS_NAMES = {0: "CP_OK", 1: "CP_ERR_INVALID_ARG", 2: "CP_ERR_UNSUPPORTED", 3: "CP_ERR_ALIGNMENT",
                 4: "CP_ERR_WORKSPACE", 5: "CP_ERR_CUDA"}
@@ -27,7 +29,7 @@ EXPORTS = [
     "cp_ring_attn_fwd_noalloc", "cp_selftest_wait_timeout", "cp_striped_reorder",
     "cp_usp_attn_workspace_size", "cp_usp_attn_fwd", "cp_ring_attn_bwd_workspace_size", "cp_ring_attn_bwd",
     "cp_usp_attn_bwd_workspace_size", "cp_usp_attn_bwd", "cp_ulysses_attn_bwd_workspace_size", "cp_ulysses_attn_bwd",
-    "cp_head_block_split",
+    "cp_head_block_split", "cp_attn_bwd_prep", "cp_block_attn_bwd",
 ]
 
 
@@ -80,6 +82,11 @@ def lib():
     L.cp_striped_reorder.argtypes = [vp, vp, i32, i32, i32, i32, i32, vp]
     L.cp_head_block_split.restype = i32
     L.cp_head_block_split.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, vp]
+    L.cp_attn_bwd_prep.restype = i32
+    L.cp_attn_bwd_prep.argtypes = [vp, vp, vp, i32, i32, i32, vp, vp, vp]
+    L.cp_block_attn_bwd.restype = i32
+    L.cp_block_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, ctypes.POINTER(cp_chunk), i32,
+                                    ctypes.POINTER(cp_chunk), i32, i32, vp, i32, f32, vp, vp, vp, i32, i32, vp]
     L.cp_zigzag_reorder.restype = i32
     L.cp_zigzag_reorder.argtypes = [vp, vp, i32, i32, i32, i32, i32, vp]
     L.cp_ulysses_attn_workspace_size.restype = i32

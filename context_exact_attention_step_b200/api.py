@@ -347,6 +347,56 @@ def ring_attn_bwd(q, k, v, o, lse, do, P, layout="contiguous", causal=True, cu_s
     return dq, dk, dv
 
 
+def attn_bwd_prep(o, lse, do, lg=None, dd=None, stream=None):
+    """Per-row vectors of the backward: lg = LSE * log2(e) (0 where LSE is
+    -inf) and dd = rowsum(dO * O), both [hq, n] fp32, from the forward's o
+    [n, hq, dh], lse [hq, n] fp32 and do [n, hq, dh] bf16 (CUDA)."""
+    _need_cuda("o", o, torch.float32)
+    _need_cuda("lse", lse, torch.float32)
+    _need_cuda("do", do, torch.bfloat16)
+    n, hq, dh = o.shape
+    if lg is None:
+        lg = torch.empty((hq, n), device=o.device, dtype=torch.float32)
+    if dd is None:
+        dd = torch.empty((hq, n), device=o.device, dtype=torch.float32)
+    check(lib().cp_attn_bwd_prep(_vp(o), _vp(do), _vp(lse), n, hq, dh, _vp(lg), _vp(dd), _stream(stream)))
+    return lg, dd
+
+
+def block_attn_bwd(q, k, v, do, lg, dd, q_chunks=None, k_chunks=None, causal=True, cu_seqlens=None,
+                   softmax_scale=0.0, dq=None, dk=None, dv=None, parts=3, accumulate=False, stream=None):
+    """Gradient contribution of one block pair: q, do [n_q, hq, dh] vs k, v
+    [n_k, hkv, dh] (bf16, CUDA), lg, dd from ``attn_bwd_prep`` of the query
+    rows; chunks and mask as ``block_attn_fwd``.  parts: 1 dQ, 2 dK/dV, 3
+    both.  accumulate: add to dq / dk / dv instead of overwriting them.
+    Returns (dq [n_q, hq, dh], dk, dv [n_k, hkv, dh]) fp32 (None for a part
+    not computed and not given)."""
+    for n, t in (("q", q), ("k", k), ("v", v), ("do", do)):
+        _need_cuda(n, t, torch.bfloat16)
+    _need_cuda("lg", lg, torch.float32)
+    _need_cuda("dd", dd, torch.float32)
+    n_q, hq, dh = q.shape
+    n_k, hkv, _ = k.shape
+    if parts & _lib.CP_BWD_DQ and dq is None:
+        dq = torch.empty((n_q, hq, dh), device=q.device, dtype=torch.float32)
+    if parts & _lib.CP_BWD_DKDV:
+        if dk is None:
+            dk = torch.empty((n_k, hkv, dh), device=q.device, dtype=torch.float32)
+        if dv is None:
+            dv = torch.empty((n_k, hkv, dh), device=q.device, dtype=torch.float32)
+    qc, nqc = _chunks(q_chunks, n_q)
+    kc, nkc = _chunks(k_chunks, n_k)
+    n_docs = 0
+    if cu_seqlens is not None:
+        _need_cuda("cu_seqlens", cu_seqlens, torch.int32)
+        n_docs = cu_seqlens.numel() - 1
+    check(lib().cp_block_attn_bwd(_vp(q), _vp(k), _vp(v), _vp(do), _vp(lg), _vp(dd), n_q, n_k, hq, hkv, dh, qc, nqc,
+                                  kc, nkc, _lib.CP_MASK_CAUSAL if causal else _lib.CP_MASK_NONE, _vp(cu_seqlens),
+                                  n_docs, float(softmax_scale), _vp(dq), _vp(dk), _vp(dv), int(parts),
+                                  1 if accumulate else 0, _stream(stream)))
+    return dq, dk, dv
+
+
 def _bwd_outputs(q, k, dq, dk, dv):
     S, hq, dh = q.shape
     hkv = k.shape[1]

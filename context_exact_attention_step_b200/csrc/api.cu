@@ -748,16 +748,19 @@ struct BwdItem {
 };
 
 // Own 128-row tiles of every rank (dq_side) or shard and every head group,
-// ordered by the number of (q, k) pairs they admit, heaviest first.
-std::vector<uint32_t> bwd_items(const cp_bwd_plan& pl, int groups, bool dq_side, const Docs& docs) {
+// ordered by the number of (q, k) pairs they admit over the plan's ring steps,
+// heaviest first.  only >= 0 keeps the tiles of that rank alone.
+std::vector<uint32_t> bwd_items(const cp_bwd_plan& pl, int groups, bool dq_side, const Docs& docs, int only = -1) {
   std::vector<BwdItem> v;
-  for (int a = 0; a < pl.P; ++a)
+  for (int a = 0; a < pl.P; ++a) {
+    if (only >= 0 && a != only) continue;
     for (int sg = 0; sg < pl.nseg[a]; ++sg) {
       const cp_seg& own = pl.seg[a][sg];
       for (int t = 0; t * 128 < own.len; ++t) {
         const int pos = own.pos + t * 128, len = std::min(128, own.len - t * 128);
         int64_t cost = 0;
-        for (int b = 0; b < pl.P; ++b)
+        for (int step = pl.t_begin; step < pl.t_end; ++step) {
+          const int b = dq_side ? ((a - step) % pl.P + pl.P) % pl.P : (a + step) % pl.P;
           for (int x = 0; x < pl.nseg[b]; ++x) {
             const cp_seg& other = pl.seg[b][x];
             // striped: a key of shard j sits one position later for rank r < j
@@ -769,10 +772,12 @@ std::vector<uint32_t> bwd_items(const cp_bwd_plan& pl, int groups, bool dq_side,
               cost += count_admitted(other.pos, other.len, pos + shift, len, pl.causal != 0, docs);
             }
           }
+        }
         for (int g = 0; g < groups; ++g)
           v.push_back({((uint32_t)a << 26) | ((uint32_t)sg << 25) | ((uint32_t)g << 19) | (uint32_t)t, cost});
       }
     }
+  }
   std::stable_sort(v.begin(), v.end(), [](const BwdItem& x, const BwdItem& y) { return x.cost > y.cost; });
   std::vector<uint32_t> out;
   out.reserve(v.size());
@@ -831,6 +836,9 @@ cp_status run_bwd(const void* qh, const void* kh, const void* vh, const void* do
   plan.dk = dk;
   plan.dv = dv;
   plan.err = err;
+  plan.t_begin = 0;
+  plan.t_end = P;
+  plan.accumulate = 0;
   Docs docs;
   if (cu_host && n_docs > 0) {
     docs.cu = cu_host;
@@ -889,6 +897,122 @@ cp_status cp_ring_attn_bwd(const void* q, const void* k, const void* v, const fl
   if ((s = run_bwd(q, k, v, dout, dout, o, lse, S, 1, hq, hkv, dh, P, layout, mask, cu_seqlens_host, cu_seqlens_dev,
                    n_docs, softmax_scale, dq, dk, dv, lg, dd, static_cast<cudaStream_t>(stream))) != CP_OK)
     return s;
+  return ok();
+}
+
+cp_status cp_attn_bwd_prep(const float* o, const void* dout, const float* lse, int n, int hq, int dh, float* lg,
+                           float* dd, void* stream) {
+  if (dh != 64 && dh != 128) return fail(CP_ERR_UNSUPPORTED, "dh = %d (supported: 64, 128)", dh);
+  if (n <= 0 || n >= (1 << 30) || hq <= 0) return fail(CP_ERR_INVALID_ARG, "n must be in [1, 2^30), hq > 0");
+  CP_CHECK_PTR(o);
+  CP_CHECK_PTR(dout);
+  CP_CHECK_PTR(lse);
+  CP_CHECK_PTR(lg);
+  CP_CHECK_PTR(dd);
+  cudaError_t e = launch_bwd_prep(dh, o, dout, lse, n, hq, 1, lg, dd, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "backward prep launch");
+  return ok();
+}
+
+// One block pair as a two-rank plan: rank 0 holds the query rows (buffer rows
+// of q, dout, dq), rank 1 the key/value rows (buffer rows of k, v, dk, dv),
+// and the ring is narrowed to step 1, at which each sees only the other.
+// Positions come from the chunks as given (a striped key shift is already
+// part of them), so the plan's striped flag stays off.
+cp_status cp_block_attn_bwd(const void* q, const void* k, const void* v, const void* dout, const float* lg,
+                            const float* dd, int n_q, int n_k, int hq, int hkv, int dh, const cp_chunk* q_chunks,
+                            int nq_chunks, const cp_chunk* k_chunks, int nk_chunks, cp_mask mask,
+                            const int32_t* cu_seqlens_dev, int n_docs, float softmax_scale, float* dq, float* dk,
+                            float* dv, int parts, int accumulate, void* stream) {
+  cp_status s;
+  if ((s = check_common(hq, hkv, dh)) != CP_OK) return s;
+  if (n_q <= 0 || n_k <= 0 || n_q >= (1 << 30) || n_k >= (1 << 30))
+    return fail(CP_ERR_INVALID_ARG, "n_q, n_k must be in [1, 2^30)");
+  if (parts < 1 || parts > (CP_BWD_DQ | CP_BWD_DKDV)) return fail(CP_ERR_INVALID_ARG, "parts = %d", parts);
+  if (accumulate != 0 && accumulate != 1) return fail(CP_ERR_INVALID_ARG, "accumulate must be 0 or 1");
+  CP_CHECK_PTR(q);
+  CP_CHECK_PTR(k);
+  CP_CHECK_PTR(v);
+  CP_CHECK_PTR(dout);
+  CP_CHECK_PTR(lg);
+  CP_CHECK_PTR(dd);
+  if (parts & CP_BWD_DQ) CP_CHECK_PTR(dq);
+  if (parts & CP_BWD_DKDV) {
+    CP_CHECK_PTR(dk);
+    CP_CHECK_PTR(dv);
+  }
+  if (mask != CP_MASK_NONE && mask != CP_MASK_CAUSAL) return fail(CP_ERR_INVALID_ARG, "unknown mask %d", (int)mask);
+  if (!q_chunks || !k_chunks) return fail(CP_ERR_INVALID_ARG, "chunk lists are NULL");
+  if (nq_chunks < 1 || nq_chunks > CP_BWD_MAX_CHUNKS || nk_chunks < 1 || nk_chunks > CP_BWD_MAX_CHUNKS)
+    return fail(CP_ERR_UNSUPPORTED, "1..%d chunks per side", CP_BWD_MAX_CHUNKS);
+  if (n_docs < 0 || (n_docs > 0 && !cu_seqlens_dev))
+    return fail(CP_ERR_INVALID_ARG, "n_docs > 0 needs cu_seqlens_dev");
+  const cp_chunk* side_chunks[2] = {q_chunks, k_chunks};
+  const int side_n[2] = {nq_chunks, nk_chunks}, side_rows[2] = {n_q, n_k};
+  cp_seg segs[2][2];
+  for (int a = 0; a < 2; ++a) {
+    int rows = 0;
+    for (int i = 0; i < side_n[a]; ++i) {
+      const cp_chunk& c = side_chunks[a][i];
+      if (c.len <= 0 || c.start < 0) return fail(CP_ERR_INVALID_ARG, "bad %s chunk %d", a ? "k" : "q", i);
+      segs[a][i] = {rows, c.start, c.len, 0};
+      rows += c.len;
+    }
+    if (rows != side_rows[a])
+      return fail(CP_ERR_INVALID_ARG, "%s chunks cover %d rows, expected %d", a ? "k" : "q", rows, side_rows[a]);
+  }
+  CUtensorMap tq, tdo, tk, tv;
+  if ((s = make_map(&tq, q, n_q, (int64_t)hq * dh, 128)) != CP_OK) return s;
+  if ((s = make_map(&tdo, dout, n_q, (int64_t)hq * dh, 128)) != CP_OK) return s;
+  if ((s = make_map(&tk, k, n_k, (int64_t)hkv * dh, 128)) != CP_OK) return s;
+  if ((s = make_map(&tv, v, n_k, (int64_t)hkv * dh, 128)) != CP_OK) return s;
+  uint32_t* err = nullptr;
+  if ((s = err_word(&err)) != CP_OK) return s;
+
+  static cp_bwd_plan plan;
+  static std::mutex plan_mu;
+  std::lock_guard<std::mutex> lk(plan_mu);
+  memset(&plan, 0, sizeof(plan));
+  plan.P = 2;
+  plan.hq = hq;
+  plan.hkv = hkv;
+  plan.causal = mask == CP_MASK_CAUSAL ? 1 : 0;
+  plan.striped = 0;
+  plan.n_docs = n_docs;
+  plan.cu_seqlens = cu_seqlens_dev;
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)dh);
+  plan.scale = scale;
+  plan.scale_log2 = scale * 1.4426950408889634f;
+  plan.S = n_q;  // row pitch of lg and dd
+  plan.group_rows = 0;
+  plan.out_hq = hq;
+  plan.out_hkv = hkv;
+  for (int a = 0; a < 2; ++a) {
+    plan.nseg[a] = side_n[a];
+    for (int i = 0; i < side_n[a]; ++i) plan.seg[a][i] = segs[a][i];
+  }
+  plan.lg = lg;
+  plan.dd = dd;
+  plan.dq = dq;
+  plan.dk = dk;
+  plan.dv = dv;
+  plan.err = err;
+  plan.t_begin = 1;
+  plan.t_end = 2;
+  plan.accumulate = accumulate;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  for (int side = 0; side < 2; ++side) {
+    const bool dq_side = side == 0;
+    if (!(parts & (dq_side ? CP_BWD_DQ : CP_BWD_DKDV))) continue;
+    const std::vector<uint32_t> items = bwd_items(plan, 1, dq_side, Docs{}, dq_side ? 0 : 1);
+    for (size_t base = 0; base < items.size(); base += CP_BWD_MAX_ITEMS) {
+      const size_t cnt = std::min(items.size() - base, (size_t)CP_BWD_MAX_ITEMS);
+      plan.n_items = (int)cnt;
+      std::copy(items.begin() + base, items.begin() + base + cnt, plan.items);
+      cudaError_t e = launch_bwd(dh, tq, tdo, tk, tv, plan, dq_side, st);
+      if (e != cudaSuccess) return cuda_fail(e, dq_side ? "block backward dQ launch" : "block backward dK/dV launch");
+    }
+  }
   return ok();
 }
 

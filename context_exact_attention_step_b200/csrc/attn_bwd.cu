@@ -26,6 +26,10 @@
 //     head of the group, and accumulates dK and dV in tensor memory.
 // No atomics: every output row is written once by one CTA.
 //
+// Across GPUs the same kernels run one block pair per launch (the plan's ring
+// steps narrowed to the one partner, and `accumulate` set so each launch adds
+// to dQ and to the dK/dV that travel with their shard).
+//
 // CTA layout of both tensor-core kernels (384 threads, one CTA per SM):
 //   warp 0      TMA producer
 //   warp 1      tcgen05.mma issuer (one elected lane) and TMEM owner
@@ -112,7 +116,8 @@ struct DqIter {
     pl = &p;
     r = own.rank;
     row0 = own.grp_row0;
-    t = sg = tl = 0;
+    t = p.t_begin;
+    sg = tl = 0;
     const int qa = own.pos0, qb = own.pos0 + own.valid - 1;
     const bool docs = p.n_docs > 0;
     vis_lo = docs ? bdoc_start(p.cu_seqlens, p.n_docs, qa) : kNoLo;
@@ -123,7 +128,7 @@ struct DqIter {
 
   __device__ bool next(KvTile& out) {
     const int P = pl->P;
-    while (t < P) {
+    while (t < pl->t_end) {
       const int j = ((r - t) % P + P) % P;
       if (sg >= pl->nseg[j]) {
         ++t;
@@ -485,6 +490,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             v.y = j > 0 ? __uint_as_float(o[4 * i + 1]) * plan.scale : 0.f;
             v.z = j > 0 ? __uint_as_float(o[4 * i + 2]) * plan.scale : 0.f;
             v.w = j > 0 ? __uint_as_float(o[4 * i + 3]) * plan.scale : 0.f;
+            if (plan.accumulate) {
+              const float4 a = d4[i];
+              v.x += a.x;
+              v.y += a.y;
+              v.z += a.z;
+              v.w += a.w;
+            }
             d4[i] = v;
           }
         }
@@ -520,7 +532,8 @@ struct KvIter {
     j = own.rank;
     hk = kv_head;
     row0 = own.grp_row0;
-    g = t = sg = tl = 0;
+    g = sg = tl = 0;
+    t = p.t_begin;
     ka0 = own.pos0;
     kb0 = own.pos0 + own.valid - 1;
     const bool docs = p.n_docs > 0;
@@ -535,9 +548,10 @@ struct KvIter {
     const int P = pl->P;
     const int group = pl->hq / pl->hkv;
     while (g < group) {
-      if (t >= P) {
+      if (t >= pl->t_end) {
         ++g;
-        t = sg = tl = 0;
+        t = pl->t_begin;
+        sg = tl = 0;
         continue;
       }
       const int r = (j + t) % P;
@@ -922,6 +936,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             v.y = i > 0 ? __uint_as_float(o[4 * k4 + 1]) * f : 0.f;
             v.z = i > 0 ? __uint_as_float(o[4 * k4 + 2]) * f : 0.f;
             v.w = i > 0 ? __uint_as_float(o[4 * k4 + 3]) * f : 0.f;
+            if (plan.accumulate) {
+              const float4 a = d4[k4];
+              v.x += a.x;
+              v.y += a.y;
+              v.z += a.z;
+              v.w += a.w;
+            }
             d4[k4] = v;
           }
         }

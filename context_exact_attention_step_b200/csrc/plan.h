@@ -120,6 +120,8 @@ struct cp_bwd_plan {
   float* dk;                    // [group_rows][out_hkv][dh]
   float* dv;                    // [group_rows][out_hkv][dh]
   uint32_t* err;
+  int32_t t_begin, t_end;       // ring steps every own tile visits: [t_begin, t_end) of 0..P-1
+  int32_t accumulate;           // 1: add to dq / dk / dv instead of overwriting them
   int32_t n_items;
   uint32_t items[CP_BWD_MAX_ITEMS];
 };

@@ -302,6 +302,56 @@ cp_status cp_ring_attn_bwd(const void* q, const void* k, const void* v, const fl
                            void* stream);
 
 /*
+ * cp_attn_bwd_prep -- the per-row vectors of the backward for n query rows:
+ *   lg[h][i] = LSE[h][i] * log2(e)  (0 where LSE = -inf: the row saw no key),
+ *   dd[h][i] = sum_c dO[i][h][c] * O[i][h][c]   (D of the gradient of softmax).
+ *   o     [n][hq][dh] fp32 and lse [hq][n] fp32: the forward's merged result
+ *   dout  [n][hq][dh] bf16, the upstream gradient
+ *   lg, dd  out, [hq][n] fp32 (caller-owned device buffers)
+ * Supported: dh in {64, 128}, 1 <= n < 2^30.  Errors: CP_ERR_INVALID_ARG /
+ * CP_ERR_ALIGNMENT for NULL or unaligned pointers; nothing launched on error.
+ *
+ * cp_block_attn_bwd -- the gradient contribution of one block pair: the
+ * query rows of one rank against one key/value shard, with the merged LSE of
+ * those query rows, i.e. one step of the ring backward of cp_ring_attn_bwd
+ * (the step a rank takes between two exchanges of the travelling K/V and
+ * dK/dV when the ranks are separate GPUs):
+ *   P  = exp(scale Q K^T - LSE) over the admitted (q, k) pairs (0 elsewhere),
+ *   dS = P * (dO V^T - D),
+ *   dq (+)= scale dS K,   dk (+)= scale dS^T Q,   dv (+)= P^T dO.
+ * The admitted pairs follow the chunk positions, mask and documents exactly as
+ * in cp_block_attn_fwd (a striped key shift belongs in k_chunks).
+ *   q, dout      [n_q][hq][dh] bf16;  k, v [n_k][hkv][dh] bf16
+ *   lg, dd       [hq][n_q] fp32 from cp_attn_bwd_prep on the same rows
+ *   q_chunks, k_chunks  host, 1..CP_BWD_MAX_CHUNKS entries per side covering
+ *                the rows in order
+ *   parts        CP_BWD_DQ, CP_BWD_DKDV or both: which outputs to compute
+ *                (the dQ kernel and the dK/dV kernel, one launch each)
+ *   accumulate   0: dq (or dk, dv) are overwritten, rows with no admitted
+ *                pair get 0; 1: the contribution is added to what they hold
+ *   dq           [n_q][hq][dh] fp32 (may be NULL without CP_BWD_DQ)
+ *   dk, dv       [n_k][hkv][dh] fp32, summed over the query heads of each KV
+ *                head (may be NULL without CP_BWD_DKDV)
+ * The pages define only the forward; this is the gradient of its exact
+ * attention, in the ring form the LSE merge of the "序列並行" concept page
+ * (compassingai), 技術原理 §二, leads to when differentiated.  No atomics:
+ * each output row is written by one CTA, so concurrent calls on different
+ * streams must not share an output buffer.  Supported: dh in {64, 128},
+ * hq % hkv == 0, 1 <= n_q, n_k < 2^30.  Errors as cp_block_attn_fwd;
+ * nothing is launched on error.
+ */
+#define CP_BWD_DQ 1
+#define CP_BWD_DKDV 2
+#define CP_BWD_MAX_CHUNKS 2
+cp_status cp_attn_bwd_prep(const float* o, const void* dout, const float* lse, int n, int hq, int dh, float* lg,
+                           float* dd, void* stream);
+cp_status cp_block_attn_bwd(const void* q, const void* k, const void* v, const void* dout, const float* lg,
+                            const float* dd, int n_q, int n_k, int hq, int hkv, int dh, const cp_chunk* q_chunks,
+                            int nq_chunks, const cp_chunk* k_chunks, int nk_chunks, cp_mask mask,
+                            const int32_t* cu_seqlens_dev, int n_docs, float softmax_scale, float* dq, float* dk,
+                            float* dv, int parts, int accumulate, void* stream);
+
+/*
  * cp_usp_attn_bwd_workspace_size / cp_usp_attn_bwd -- gradients of
  * cp_usp_attn_fwd (the Ulysses-inside / Ring-across hybrid) for an upstream
  * gradient dO, with the same rank grid, layouts and support as the forward.

@@ -367,7 +367,6 @@ def ring_attention_bwd(q, k, v, do, S, P, layout, causal=True, cu_seqlens=None, 
     do = np.asarray(do, dtype=np.float64)
     hq, dh = q.shape[1], q.shape[2]
     hkv = k.shape[1]
-    group = hq // hkv
     if scale is None:
         scale = 1.0 / math.sqrt(dh)
     o_all, lse_all = ring_attention(q, k, v, S, P, layout, causal, cu_seqlens, scale)
@@ -382,18 +381,46 @@ def ring_attention_bwd(q, k, v, do, S, P, layout, causal=True, cu_seqlens=None, 
             qp, kp = pos[r], pos[j]
             o_r = o_all[r * n:(r + 1) * n]
             lse_r = lse_all[:, r * n:(r + 1) * n]
-            mask = explicit_mask(qp, kp, causal, cu_seqlens)
-            for h in range(hq):
-                g = h // group
-                s = (q[qp, h, :] @ k[kp, g, :].T) * scale
-                lse_h = np.where(np.isfinite(lse_r[h]), lse_r[h], 0.0)
-                p = np.where(mask, np.exp(s - lse_h[:, None]), 0.0)
-                d = (do[qp, h, :] * o_r[:, h, :]).sum(axis=1)
-                ds = p * (do[qp, h, :] @ v[kp, g, :].T - d[:, None])
-                dq[r][:, h, :] += scale * (ds @ k[kp, g, :])
-                dk[j][:, g, :] += scale * (ds.T @ q[qp, h, :])
-                dv[j][:, g, :] += p.T @ do[qp, h, :]
+            gq, gk, gv = ring_pair_bwd(q[qp], k[kp], v[kp], do[qp], o_r, lse_r, qp, kp, causal, cu_seqlens, scale)
+            dq[r] += gq
+            dk[j] += gk
+            dv[j] += gv
     return np.concatenate(dq), np.concatenate(dk), np.concatenate(dv)
+
+
+def ring_pair_bwd(q_r, k_j, v_j, do_r, o_r, lse_r, qpos, kpos, causal=True, cu_seqlens=None, scale=None,
+                  d_r=None):
+    """One ring step of the backward: the contributions of block pair (r, j)
+    to dQ_r, dK_j and dV_j, from rank r's rows q_r, do_r [n_q, Hq, dh], its
+    merged forward o_r [n_q, Hq, dh] and lse_r [Hq, n_q], and shard j's k_j,
+    v_j [n_k, Hkv, dh]; qpos, kpos are the rows' global positions.  With
+    P_rj = exp(scale Q_r K_j^T - LSE_r) on the admitted pairs and
+    D_r = rowsum(dO_r * O_r):  dS = P_rj * (dO_r V_j^T - D_r),
+    dQ = scale dS K_j, dK = scale dS^T Q_r, dV = P_rj^T dO_r (GQA: summed over
+    the query heads of each KV head).  d_r [Hq, n_q], when given, is D_r
+    itself and o_r is not read."""
+    q_r, k_j, v_j, do_r, lse_r = (np.asarray(a, dtype=np.float64) for a in (q_r, k_j, v_j, do_r, lse_r))
+    if d_r is None:
+        d_r = (do_r * np.asarray(o_r, dtype=np.float64)).sum(axis=2).T
+    d_r = np.asarray(d_r, dtype=np.float64)
+    hq, dh = q_r.shape[1], q_r.shape[2]
+    group = hq // k_j.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(dh)
+    mask = explicit_mask(np.asarray(qpos), np.asarray(kpos), causal, cu_seqlens)
+    dq = np.zeros(q_r.shape)
+    dk = np.zeros(k_j.shape)
+    dv = np.zeros(v_j.shape)
+    for h in range(hq):
+        g = h // group
+        s = (q_r[:, h, :] @ k_j[:, g, :].T) * scale
+        lse_h = np.where(np.isfinite(lse_r[h]), lse_r[h], 0.0)
+        p = np.where(mask, np.exp(s - lse_h[:, None]), 0.0)
+        ds = p * (do_r[:, h, :] @ v_j[:, g, :].T - d_r[h][:, None])
+        dq[:, h, :] += scale * (ds @ k_j[:, g, :])
+        dk[:, g, :] += scale * (ds.T @ q_r[:, h, :])
+        dv[:, g, :] += p.T @ do_r[:, h, :]
+    return dq, dk, dv
 
 
 def live_pair_count(S, causal=True, cu_seqlens=None, qpos=None, kpos=None):

@@ -26,3 +26,18 @@ def compare(o_gpu, lse_gpu, o_ref, lse_ref, o_tol=O_TOL, lse_tol=LSE_TOL, what="
     assert err_o <= o_tol, f"{what}: O max-abs error {err_o:.3e} > {o_tol}"
     assert err_l <= lse_tol, f"{what}: LSE max-abs error {err_l:.3e} > {lse_tol}"
     return err_o, err_l
+
+
+# gradients: relative to the largest entry of the reference tensor (the
+# derivation of 2e-2 sits with the backward parity tests)
+GRAD_REL_TOL = 2e-2
+
+
+def check_grad(got, want, what, rel_tol=GRAD_REL_TOL):
+    got = f64(got) if isinstance(got, torch.Tensor) else got
+    assert got.shape == want.shape, (what, got.shape, want.shape)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite"
+    scale = float(np.max(np.abs(want))) if want.size else 0.0
+    err = float(np.max(np.abs(got - want))) if want.size else 0.0
+    assert err <= rel_tol * max(scale, 1e-6), f"{what}: max-abs error {err:.3e} vs max |ref| {scale:.3e}"
+    return err / max(scale, 1e-30)

@@ -150,6 +150,36 @@ def test_ring_bwd_workspace_is_two_vectors_per_head():
     assert api.ring_attn_bwd_workspace_size(4096, 32, 8, 128, 4, "zigzag") == 2 * a(4096 * 32 * 4)
 
 
+def _pair_bwd(n_q=256, n_k=256, hq=4, hkv=2, dh=128, qc=((0, 256),), kc=((0, 256),), parts=3, acc=0, dq=FAKE,
+              dk=FAKE, lg=FAKE, mask=_lib.CP_MASK_CAUSAL, n_docs=0):
+    qa = (_lib.cp_chunk * len(qc))(*[_lib.cp_chunk(a, b) for a, b in qc])
+    ka = (_lib.cp_chunk * len(kc))(*[_lib.cp_chunk(a, b) for a, b in kc])
+    return lib().cp_block_attn_bwd(FAKE, FAKE, FAKE, FAKE, lg, FAKE, n_q, n_k, hq, hkv, dh, qa, len(qc), ka, len(kc),
+                                   mask, ctypes.c_void_p(0), n_docs, 0.0, dq, dk, FAKE, parts, acc,
+                                   ctypes.c_void_p(0))
+
+
+def test_block_bwd_rejects_bad_arguments():
+    assert _pair_bwd(dh=96) == _lib.CP_ERR_UNSUPPORTED
+    assert _pair_bwd(hq=3) == _lib.CP_ERR_INVALID_ARG
+    assert _pair_bwd(n_q=0) == _lib.CP_ERR_INVALID_ARG
+    assert _pair_bwd(parts=0) == _lib.CP_ERR_INVALID_ARG
+    assert _pair_bwd(parts=4) == _lib.CP_ERR_INVALID_ARG
+    assert _pair_bwd(acc=2) == _lib.CP_ERR_INVALID_ARG
+    assert _pair_bwd(dq=ctypes.c_void_p(0)) == _lib.CP_ERR_INVALID_ARG          # dQ asked for, no buffer
+    assert _pair_bwd(dk=ctypes.c_void_p(0)) == _lib.CP_ERR_INVALID_ARG          # dK/dV asked for, no buffer
+    assert _pair_bwd(lg=MISALIGNED) == _lib.CP_ERR_ALIGNMENT
+    assert _pair_bwd(mask=7) == _lib.CP_ERR_INVALID_ARG
+    assert _pair_bwd(qc=((0, 100), (200, 100), (400, 56))) == _lib.CP_ERR_UNSUPPORTED  # three chunks
+    assert _pair_bwd(qc=((0, 100),)) == _lib.CP_ERR_INVALID_ARG                 # chunks miss rows
+    assert _pair_bwd(kc=((-1, 256),)) == _lib.CP_ERR_INVALID_ARG
+    assert _pair_bwd(n_docs=2) == _lib.CP_ERR_INVALID_ARG                       # documents without the table
+    L = lib()
+    assert L.cp_attn_bwd_prep(FAKE, FAKE, FAKE, 128, 4, 96, FAKE, FAKE, None) == _lib.CP_ERR_UNSUPPORTED
+    assert L.cp_attn_bwd_prep(FAKE, FAKE, FAKE, 0, 4, 128, FAKE, FAKE, None) == _lib.CP_ERR_INVALID_ARG
+    assert L.cp_attn_bwd_prep(FAKE, FAKE, FAKE, 128, 4, 128, FAKE, ctypes.c_void_p(0), None) == _lib.CP_ERR_INVALID_ARG
+
+
 def test_permute_and_merge_reject_bad_arguments():
     L = lib()
     # Ulysses head limit: P must divide the head count

@@ -1,12 +1,14 @@
 """Multi-process (gloo, CPU) tests of the communication in
 ``context_exact_attention_step_b200.distributed``: the ring's K/V rotation
-with live-step skipping and the two Ulysses all-to-alls, on 2 and 4 ranks.
+with live-step skipping and the two Ulysses all-to-alls, forward and
+backward (where the shard's dK/dV travel with it), on 2, 3 and 4 ranks.
 
 The library's CUDA kernels cannot run here, so each rank passes stand-ins
-with the same signatures: the fp64 oracle for block attention and the LSE
-merge, a reshape for the head-block split, and the library's own host
-scheduler for the skip decisions.  Every rank's result must equal the oracle's
-attention over the whole sequence for that rank's rows."""
+with the same signatures: the fp64 oracle for block attention, the block
+pair's backward and the LSE merge, a reshape for the head-block split, and
+the library's own host scheduler for the skip decisions.  Every rank's result
+must equal the oracle's attention (or its gradient) over the whole sequence
+for that rank's rows."""
 import os
 import socket
 import sys
@@ -53,6 +55,40 @@ class OracleKernels:
         return torch.from_numpy(o), torch.from_numpy(lse)
 
     @staticmethod
+    def attn_bwd_prep(o, lse, do):
+        # the stand-in's per-row state: the merged LSE itself and D = rowsum(dO * O)
+        return lse.clone(), (do * o).sum(dim=2).T.contiguous()
+
+    @staticmethod
+    def block_attn_bwd(q, k, v, do, lg, dd, q_chunks, k_chunks, causal, cu_dev, scale, dq=None, dk=None, dv=None,
+                       parts=3, accumulate=False):
+        from oracle import ref
+        qpos = np.concatenate([np.arange(a, a + n) for a, n in q_chunks])
+        kpos = np.concatenate([np.arange(a, a + n) for a, n in k_chunks])
+        cu = None if cu_dev is None else cu_dev.tolist()
+        grads = ref.ring_pair_bwd(q.numpy(), k.numpy(), v.numpy(), do.numpy(), None, lg.numpy(), qpos, kpos, causal,
+                                  cu, scale or None, d_r=dd.numpy())
+        for g, out, bit in zip(grads, (dq, dk, dv), (1, 2, 2)):
+            if parts & bit:
+                t = torch.from_numpy(g).to(out.dtype)
+                if accumulate:
+                    out += t
+                else:
+                    out.copy_(t)
+        return dq, dk, dv
+
+    @staticmethod
+    def ring_attn_bwd(q, k, v, o, lse, do, P, layout, causal, softmax_scale=0.0):
+        # the head-layout backward over the whole sequence, from the O and LSE
+        # it is given (so their transposes are checked too)
+        from oracle import ref
+        assert P == 1 and layout == "contiguous"
+        pos = np.arange(q.shape[0])
+        grads = ref.ring_pair_bwd(q.numpy(), k.numpy(), v.numpy(), do.numpy(), o.numpy(), lse.numpy(), pos, pos,
+                                  causal, None, softmax_scale or None)
+        return tuple(torch.from_numpy(g) for g in grads)
+
+    @staticmethod
     def head_block_split(x, P, inverse=False):
         if not inverse:
             n, h, dh = x.shape
@@ -76,9 +112,23 @@ def _worker(rank, world, port, kind, cfg, results):
         if kind == "ring":
             o, lse = D.ring_attn_fwd_dist(q[idx], k[idx], v[idx], layout, cfg["causal"], cfg.get("cu"),
                                           kernels=OracleKernels)
-        else:
+            results[rank] = (o.numpy(), lse.numpy())
+        elif kind == "ulysses":
             o, lse = D.ulysses_attn_fwd_dist(q[idx], k[idx], v[idx], cfg["causal"], kernels=OracleKernels)
-        results[rank] = (o.numpy(), lse.numpy())
+            results[rank] = (o.numpy(), lse.numpy())
+        else:
+            # the forward's merged O and LSE of this rank's rows, from the oracle
+            do = synth.normal((S, hq, dh), synth.SEED_DO, 0.5).double()
+            o_all, lse_all = ref.attention(q.numpy(), k.numpy(), v.numpy(), causal=cfg["causal"],
+                                           cu_seqlens=cfg.get("cu"))
+            o, lse = torch.from_numpy(o_all[rows]), torch.from_numpy(np.ascontiguousarray(lse_all[:, rows]))
+            if kind == "ring_bwd":
+                grads = D.ring_attn_bwd_dist(q[idx], k[idx], v[idx], o, lse, do[idx], layout, cfg["causal"],
+                                             cfg.get("cu"), kernels=OracleKernels)
+            else:
+                grads = D.ulysses_attn_bwd_dist(q[idx], k[idx], v[idx], o, lse, do[idx], cfg["causal"],
+                                                kernels=OracleKernels)
+            results[rank] = tuple(g.numpy() for g in grads)
     finally:
         dist.destroy_process_group()
 
@@ -91,6 +141,14 @@ def _run(kind, world, cfg):
     mp.spawn(_worker, args=(world, _free_port(), kind, cfg, results), nprocs=world, join=True)
     S, hq, hkv, dh = cfg["S"], cfg["hq"], cfg["hkv"], cfg["dh"]
     q, k, v = (t.double().numpy() for t in synth.qkv(S, hq, hkv, dh))
+    if kind.endswith("_bwd"):
+        do = synth.normal((S, hq, dh), synth.SEED_DO, 0.5).double().numpy()
+        want = ref.attention_bwd(q, k, v, do, causal=cfg["causal"], cu_seqlens=cfg.get("cu"))
+        for r in range(world):
+            rows = ref.shard_positions(S, world, cfg.get("layout", "contiguous"), r)
+            for got, w, what in zip(results[r], want, ("dQ", "dK", "dV")):
+                np.testing.assert_allclose(got, w[rows], atol=1e-10, err_msg=f"{what} of rank {r}")
+        return
     want_o, want_l = ref.attention(q, k, v, causal=cfg["causal"], cu_seqlens=cfg.get("cu"))
     for r in range(world):
         rows = ref.shard_positions(S, world, cfg.get("layout", "contiguous"), r)
@@ -122,3 +180,27 @@ def test_ulysses_over_ranks(world):
 
 def test_ulysses_over_ranks_noncausal():
     _run("ulysses", 2, dict(S=32, hq=4, hkv=2, dh=8, causal=False))
+
+
+@pytest.mark.parametrize("layout,world", [("contiguous", 2), ("zigzag", 4), ("striped", 2), ("striped", 4)])
+def test_ring_bwd_over_ranks(layout, world):
+    _run("ring_bwd", world, dict(S=64, hq=4, hkv=2, dh=8, layout=layout, causal=True))
+
+
+def test_ring_bwd_over_three_ranks_documents():
+    # an odd ring with documents: some steps are skipped, yet every shard's
+    # gradient still makes the full circle home
+    _run("ring_bwd", 3, dict(S=48, hq=2, hkv=1, dh=8, layout="zigzag", causal=True, cu=[0, 7, 8, 30, 48]))
+
+
+def test_ring_bwd_over_ranks_noncausal():
+    _run("ring_bwd", 2, dict(S=32, hq=2, hkv=2, dh=8, layout="contiguous", causal=False))
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_ulysses_bwd_over_ranks(world):
+    _run("ulysses_bwd", world, dict(S=32, hq=8, hkv=4, dh=8, causal=True))
+
+
+def test_ulysses_bwd_over_ranks_noncausal():
+    _run("ulysses_bwd", 2, dict(S=32, hq=4, hkv=2, dh=8, causal=False))

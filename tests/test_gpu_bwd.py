@@ -13,27 +13,18 @@ import pytest
 import torch
 
 from context_exact_attention_step_b200 import api, synth
+from context_exact_attention_step_b200 import distributed as D
 from oracle import ref
 
-from _util import f64
+from _util import GRAD_REL_TOL, check_grad, f64
 
 pytestmark = pytest.mark.gpu
 
-REL_TOL = 2e-2
+assert GRAD_REL_TOL == 2e-2
 
 
 def storage_order(S, P, layout):
     return np.concatenate([ref.shard_positions(S, P, layout, r) for r in range(P)])
-
-
-def check_grad(got, want, what):
-    got = f64(got)
-    assert got.shape == want.shape, (what, got.shape, want.shape)
-    assert np.all(np.isfinite(got)), f"{what}: non-finite"
-    scale = float(np.max(np.abs(want)))
-    err = float(np.max(np.abs(got - want)))
-    assert err <= REL_TOL * max(scale, 1e-6), f"{what}: max-abs error {err:.3e} vs max |ref| {scale:.3e}"
-    return err / max(scale, 1e-30)
 
 
 def bwd_case(S, hq, hkv, dh, P, layout, causal=True, cu=None):
@@ -217,3 +208,102 @@ def test_bwd_gqa_documents():
     S = 2048
     lens = synth.doc_lengths(S, 50, 600, seed=10)
     bwd_case(S, 8, 2, 64, 4, "zigzag", cu=synth.cu_seqlens_from_lengths(lens).tolist())
+
+
+# ------------------------------------------- block pairs: one step of the ring across GPUs
+def _pair_setup(S, hq, hkv, dh, P, layout, causal, cu):
+    q, k, v = synth.qkv(S, hq, hkv, dh)
+    do = synth.normal((S, hq, dh), synth.SEED_DO, 0.5)
+    o_ref, lse_ref = ref.attention(f64(q), f64(k), f64(v), causal=causal, cu_seqlens=cu)
+    return q, k, v, do, o_ref, lse_ref
+
+
+@pytest.mark.parametrize("layout,r,j", [("zigzag", 1, 3), ("zigzag", 3, 0), ("contiguous", 2, 2),
+                                        ("striped", 1, 2), ("striped", 2, 1)])
+def test_block_bwd_pair(layout, r, j):
+    # the rows of rank r against shard j, with the merged O and LSE of the
+    # whole attention: equal to the oracle's contribution of that pair
+    S, hq, hkv, dh, P = 2048, 4, 2, 128, 4
+    q, k, v, do, o_ref, lse_ref = _pair_setup(S, hq, hkv, dh, P, layout, True, None)
+    qp, kp = ref.shard_positions(S, P, layout, r), ref.shard_positions(S, P, layout, j)
+    qi, ki = torch.from_numpy(qp), torch.from_numpy(kp)
+    o_r = torch.from_numpy(o_ref[qp]).float().cuda()
+    lse_r = torch.from_numpy(np.ascontiguousarray(lse_ref[:, qp])).float().cuda()
+    q_r, do_r = q[qi].contiguous().cuda(), do[qi].contiguous().cuda()
+    k_j, v_j = k[ki].contiguous().cuda(), v[ki].contiguous().cuda()
+    lg, dd = api.attn_bwd_prep(o_r, lse_r, do_r)
+    qc, kc = D.query_chunks(S, P, layout, r), D.key_chunks(S, P, layout, r, j)
+    dq, dk, dv = api.block_attn_bwd(q_r, k_j, v_j, do_r, lg, dd, qc, kc, True)
+    torch.cuda.synchronize()
+    assert api.device_error() == 0
+    want = ref.ring_pair_bwd(f64(q)[qp], f64(k)[kp], f64(v)[kp], f64(do)[qp], o_ref[qp], lse_ref[:, qp], qp, kp,
+                             causal=True)
+    for got, w, what in zip((dq, dk, dv), want, ("dQ", "dK", "dV")):
+        if np.max(np.abs(w)) == 0.0:
+            assert float(got.abs().max()) == 0.0, f"{what}: a pair with no admitted keys must give 0"
+        else:
+            check_grad(got, w, f"{what} {layout} r={r} j={j}")
+
+
+def test_block_bwd_parts_and_accumulate():
+    # parts picks the kernels; accumulate adds to what the buffers hold
+    S, hq, hkv, dh = 640, 2, 2, 64
+    q, k, v, do, o_ref, lse_ref = _pair_setup(S, hq, hkv, dh, 1, "contiguous", False, None)
+    qd, kd, vd, dod = (t.cuda() for t in (q, k, v, do))
+    o = torch.from_numpy(o_ref).float().cuda()
+    lse = torch.from_numpy(lse_ref).float().cuda()
+    lg, dd = api.attn_bwd_prep(o, lse, dod)
+    base_q = torch.randn(S, hq, dh, device="cuda")
+    base_k = torch.randn(S, hkv, dh, device="cuda")
+    dq = base_q.clone()
+    dk, dv = base_k.clone(), base_k.clone()
+    api.block_attn_bwd(qd, kd, vd, dod, lg, dd, causal=False, dq=dq, parts=1, accumulate=True)
+    torch.cuda.synchronize()
+    assert torch.equal(dk, base_k) and torch.equal(dv, base_k), "parts=1 must leave dK, dV alone"
+    api.block_attn_bwd(qd, kd, vd, dod, lg, dd, causal=False, dk=dk, dv=dv, parts=2, accumulate=True)
+    torch.cuda.synchronize()
+    assert api.device_error() == 0
+    wq, wk, wv = ref.attention_bwd(f64(q), f64(k), f64(v), f64(do), causal=False)
+    check_grad(f64(dq) - f64(base_q), wq, "accumulated dQ")
+    check_grad(f64(dk) - f64(base_k), wk, "accumulated dK")
+    check_grad(f64(dv) - f64(base_k), wv, "accumulated dV")
+
+
+@pytest.mark.parametrize("layout", ["contiguous", "zigzag", "striped"])
+def test_block_bwd_ring_emulated(layout):
+    # the multi-GPU ring backward's arithmetic on one GPU: for every ring step
+    # and rank, one block-pair call adding to dQ_r and to the dK_j, dV_j the
+    # shard carries; the sums must equal the gradient of the whole attention
+    S, hq, hkv, dh, P = 2048, 4, 2, 64, 4
+    lens = synth.doc_lengths(S, 64, 900, seed=12)
+    cu = synth.cu_seqlens_from_lengths(lens).tolist()
+    if layout == "striped":
+        cu = None  # the striped layout has no document mask
+    q, k, v, do, o_ref, lse_ref = _pair_setup(S, hq, hkv, dh, P, layout, True, cu)
+    sched = api.ring_schedule(S, P, layout, True, cu)
+    cu_dev = None if cu is None else torch.tensor(cu, dtype=torch.int32, device="cuda")
+    pos = [ref.shard_positions(S, P, layout, r) for r in range(P)]
+    take = lambda t, r: t[torch.from_numpy(pos[r])].contiguous().cuda()
+    qs, ks, vs, dos = ([take(t, r) for r in range(P)] for t in (q, k, v, do))
+    preps = [api.attn_bwd_prep(torch.from_numpy(o_ref[pos[r]]).float().cuda(),
+                               torch.from_numpy(np.ascontiguousarray(lse_ref[:, pos[r]])).float().cuda(), dos[r])
+             for r in range(P)]
+    n = S // P
+    dq = [torch.empty(n, hq, dh, device="cuda") for _ in range(P)]
+    dk = [torch.empty(n, hkv, dh, device="cuda") for _ in range(P)]
+    dv = [torch.empty(n, hkv, dh, device="cuda") for _ in range(P)]
+    for t in range(P):
+        for r in range(P):
+            j = (r - t) % P
+            assert sched["launched"][r * P + t] or t > 0
+            if sched["launched"][r * P + t]:
+                api.block_attn_bwd(qs[r], ks[j], vs[j], dos[r], *preps[r], D.query_chunks(S, P, layout, r),
+                                   D.key_chunks(S, P, layout, r, j), True, cu_dev, dq=dq[r], dk=dk[j], dv=dv[j],
+                                   accumulate=t > 0)
+    torch.cuda.synchronize()
+    assert api.device_error() == 0
+    wq, wk, wv = ref.attention_bwd(f64(q), f64(k), f64(v), f64(do), causal=True, cu_seqlens=cu)
+    order = storage_order(S, P, layout)
+    check_grad(torch.cat(dq), wq[order], f"emulated ring dQ {layout}")
+    check_grad(torch.cat(dk), wk[order], f"emulated ring dK {layout}")
+    check_grad(torch.cat(dv), wv[order], f"emulated ring dV {layout}")

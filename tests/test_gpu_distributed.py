@@ -4,7 +4,6 @@ exchanges themselves are covered by the multi-rank gloo tests."""
 import os
 import socket
 
-import numpy as np
 import pytest
 import torch
 import torch.distributed as dist
@@ -12,7 +11,7 @@ import torch.distributed as dist
 from context_exact_attention_step_b200 import distributed as D, synth
 from oracle import ref
 
-from _util import compare, f64
+from _util import check_grad, compare, f64
 
 pytestmark = pytest.mark.gpu
 
@@ -45,3 +44,29 @@ def test_ulysses_dist_one_rank(one_rank_group):
     torch.cuda.synchronize()
     want_o, want_l = ref.attention(f64(q), f64(k), f64(v), causal=False)
     compare(o, lse, want_o, want_l, what="ulysses over one rank")
+
+
+def test_ring_bwd_dist_one_rank(one_rank_group):
+    S, hq, hkv, dh = 1024, 4, 2, 128
+    q, k, v = synth.qkv(S, hq, hkv, dh)
+    do = synth.normal((S, hq, dh), synth.SEED_DO, 0.5)
+    qd, kd, vd, dod = (t.cuda() for t in (q, k, v, do))
+    o, lse = D.ring_attn_fwd_dist(qd, kd, vd, "contiguous", True)
+    dq, dk, dv = D.ring_attn_bwd_dist(qd, kd, vd, o, lse, dod, "contiguous", True)
+    torch.cuda.synchronize()
+    want = ref.attention_bwd(f64(q), f64(k), f64(v), f64(do), causal=True)
+    for got, w, what in zip((dq, dk, dv), want, ("dQ", "dK", "dV")):
+        check_grad(got, w, f"ring backward over one rank: {what}")
+
+
+def test_ulysses_bwd_dist_one_rank(one_rank_group):
+    S, hq, hkv, dh = 1024, 4, 2, 64
+    q, k, v = synth.qkv(S, hq, hkv, dh)
+    do = synth.normal((S, hq, dh), synth.SEED_DO, 0.5)
+    qd, kd, vd, dod = (t.cuda() for t in (q, k, v, do))
+    o, lse = D.ulysses_attn_fwd_dist(qd, kd, vd, False)
+    dq, dk, dv = D.ulysses_attn_bwd_dist(qd, kd, vd, o, lse, dod, False)
+    torch.cuda.synchronize()
+    want = ref.attention_bwd(f64(q), f64(k), f64(v), f64(do), causal=False)
+    for got, w, what in zip((dq, dk, dv), want, ("dQ", "dK", "dV")):
+        check_grad(got, w, f"ulysses backward over one rank: {what}")

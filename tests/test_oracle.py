@@ -444,6 +444,26 @@ def test_ring_bwd_with_documents_equals_unsplit():
         np.testing.assert_allclose(a, b[order], atol=1e-12)
 
 
+def test_ring_pair_bwd_single_pair_is_whole_gradient_and_takes_d():
+    # one pair covering every row and key is the whole gradient (pinned
+    # against autograd above); passing D = rowsum(dO * O) directly changes
+    # nothing; a pair that admits no (q, k) gives exactly zero
+    S, hq, hkv, dh = 24, 4, 2, 8
+    q, k, v, do = randn(S, hq, dh), randn(S, hkv, dh), randn(S, hkv, dh), randn(S, hq, dh)
+    o, lse = ref.attention(q, k, v, causal=True)
+    pos = np.arange(S)
+    want = ref.attention_bwd(q, k, v, do, causal=True)
+    got = ref.ring_pair_bwd(q, k, v, do, o, lse, pos, pos, causal=True)
+    d = np.einsum("shc,shc->hs", do, o)
+    got_d = ref.ring_pair_bwd(q, k, v, do, None, lse, pos, pos, causal=True, d_r=d)
+    for a, b, c in zip(got, got_d, want):
+        np.testing.assert_allclose(a, c, atol=1e-12)
+        np.testing.assert_allclose(a, b, atol=1e-13)  # D summed in another order
+    # queries 0..7 against keys 16..23 under causal: nothing admitted
+    zero = ref.ring_pair_bwd(q[:8], k[16:], v[16:], do[:8], o[:8], lse[:, :8], pos[:8], pos[16:], causal=True)
+    assert all(not np.any(z) for z in zero)
+
+
 # ------------------------------------------------------ work counts
 def test_live_pair_counts_closed_forms():
     S = 96

@@ -21,6 +21,10 @@ shard r of the sequence in the same order the single-GPU entry points use
   of its own heads, it attends over the whole sequence, and a second
   all-to-all plus the inverse regrouping bring O back to sequence shards.
 
+* USP (compassingai, closing section: Ulysses inside the NVLink domain, Ring
+  across it; pwwt.cn §6): a Pr x Pu grid of ranks, Ulysses inside each group
+  of Pu ranks, then a ring over the Pr groups for every head block, each on
+  its own process group (``usp_groups``).
 * Backward (the gradient of the same exact attention; the pages define the
   forward only): the ring form keeps each rank's merged O and LSE, so at step
   t rank r adds the contribution of block pair (r, j) to its dQ_r and to the
@@ -114,6 +118,45 @@ def ring_attn_fwd_dist(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, layout
     return kernels.lse_merge(parts_o, parts_l)
 
 
+def _seq_to_heads(x: torch.Tensor, P: int, group, kernels) -> torch.Tensor:
+    """[n, h, dh] rows of this rank -> [P*n, h/P, dh]: every rank's rows of
+    this rank's head block (block p of the heads goes to rank p)."""
+    n, h, dh = x.shape
+    blocks = kernels.head_block_split(x, P)           # [P, n, h/P, dh]: block p goes to rank p
+    got = torch.empty_like(blocks)
+    dist.all_to_all_single(got, blocks, group=group)  # got[p] = rank p's rows of my heads
+    return got.view(P * n, h // P, dh)
+
+
+def _heads_to_seq(x_h: torch.Tensor, P: int, group, kernels) -> torch.Tensor:
+    """Inverse of _seq_to_heads: [P*n, hb, dh] -> [n, P*hb, dh]."""
+    rows, hb, dh = x_h.shape
+    n = rows // P
+    blocks = torch.empty_like(x_h).view(P, n, hb, dh)
+    dist.all_to_all_single(blocks, x_h.view(P, n, hb, dh).contiguous(), group=group)
+    return kernels.head_block_split(blocks, P, inverse=True)
+
+
+def _lse_seq_to_heads(lse: torch.Tensor, P: int, group, kernels) -> torch.Tensor:
+    """LSE [h, n] of this rank's rows -> [h/P, P*n] of its head block: head
+    block p goes to rank p, and the [P][h/P][n] slabs received become
+    [h/P][P][n]."""
+    h, n = lse.shape
+    got = torch.empty_like(lse)
+    dist.all_to_all_single(got, lse.contiguous(), group=group)
+    return kernels.head_block_split(got.view(P, h // P, 1, n), P, inverse=True).view(h // P, P * n)
+
+
+def _lse_heads_to_seq(lse_h: torch.Tensor, P: int, group, kernels) -> torch.Tensor:
+    """Inverse of _lse_seq_to_heads: [hb, P*n] -> [P*hb, n]."""
+    hb, rows = lse_h.shape
+    n = rows // P
+    send = kernels.head_block_split(lse_h.view(hb, P, n), P).view(P, hb, n)  # slab p: rank p's rows
+    got = torch.empty_like(send)
+    dist.all_to_all_single(got, send.contiguous(), group=group)
+    return got.view(P * hb, n)
+
+
 def ulysses_attn_fwd_dist(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = True, group=None,
                           softmax_scale: float = 0.0, kernels=_api):
     """DeepSpeed-Ulysses forward over the ranks of ``group``.  q [n, hq, dh],
@@ -121,30 +164,13 @@ def ulysses_attn_fwd_dist(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cau
     r*n .. r*n + n - 1).  P must divide hkv (no KV replication).
     Returns this rank's (O [n, hq, dh] fp32, LSE [hq, n] fp32)."""
     P = dist.get_world_size(group)
-    n, hq, dh = q.shape
-    hkv = k.shape[1]
-    if hkv % P != 0:
-        raise ValueError(f"P = {P} must divide the KV head count {hkv}")
+    n = q.shape[0]
+    if k.shape[1] % P != 0:
+        raise ValueError(f"P = {P} must divide the KV head count {k.shape[1]}")
     S = n * P
-    hg = hq // P
-
-    def to_heads(x):
-        blocks = kernels.head_block_split(x, P)           # [P, n, h/P, dh]: block p goes to rank p
-        got = torch.empty_like(blocks)
-        dist.all_to_all_single(got, blocks, group=group)  # got[p] = rank p's rows of my heads
-        return got.view(S, x.shape[1] // P, dh)
-
-    qh, kh, vh = to_heads(q), to_heads(k), to_heads(v)
+    qh, kh, vh = (_seq_to_heads(x, P, group, kernels) for x in (q, k, v))
     o_h, lse_h = kernels.block_attn_fwd(qh, kh, vh, [(0, S)], [(0, S)], causal, None, softmax_scale)
-    # O back to sequence shards: block p of my heads' output holds rank p's rows
-    o_blocks = torch.empty_like(o_h).view(P, n, hg, dh)
-    dist.all_to_all_single(o_blocks, o_h.view(P, n, hg, dh).contiguous(), group=group)
-    o = kernels.head_block_split(o_blocks, P, inverse=True)  # [n, hq, dh]
-    # LSE [hg, S] -> per destination rank p the [hg, n] slab of its rows
-    lse_send = kernels.head_block_split(lse_h.view(hg, P, n), P).view(P, hg, n)
-    lse_recv = torch.empty_like(lse_send)
-    dist.all_to_all_single(lse_recv, lse_send.contiguous(), group=group)
-    return o, lse_recv.view(hq, n)
+    return _heads_to_seq(o_h, P, group, kernels), _lse_heads_to_seq(lse_h, P, group, kernels)
 
 
 def ring_attn_bwd_dist(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse: torch.Tensor,
@@ -219,31 +245,71 @@ def ulysses_attn_bwd_dist(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: 
     upstream do [n, hq, dh].  Returns this rank's (dQ [n, hq, dh], dK, dV
     [n, hkv, dh]) fp32."""
     P = dist.get_world_size(group)
-    n, hq, dh = q.shape
-    hkv = k.shape[1]
-    if hkv % P != 0:
-        raise ValueError(f"P = {P} must divide the KV head count {hkv}")
-    S = n * P
-    hg = hq // P
-
-    def to_heads(x):
-        blocks = kernels.head_block_split(x, P)
-        got = torch.empty_like(blocks)
-        dist.all_to_all_single(got, blocks, group=group)
-        return got.view(S, x.shape[1] // P, x.shape[2])
-
-    def to_seq(x_h):
-        h = x_h.shape[1]
-        blocks = torch.empty_like(x_h).view(P, n, h, dh)
-        dist.all_to_all_single(blocks, x_h.view(P, n, h, dh).contiguous(), group=group)
-        return kernels.head_block_split(blocks, P, inverse=True)
-
-    qh, kh, vh, doh, oh = (to_heads(x) for x in (q, k, v, do, o))
-    # LSE [hq, n]: head block p goes to rank p; the [P][hg][n] slabs received
-    # become [hg][P][n] = [hg, S]
-    lse_recv = torch.empty_like(lse)
-    dist.all_to_all_single(lse_recv, lse.contiguous(), group=group)
-    lse_h = kernels.head_block_split(lse_recv.view(P, hg, 1, n), P, inverse=True).view(hg, S)
+    if k.shape[1] % P != 0:
+        raise ValueError(f"P = {P} must divide the KV head count {k.shape[1]}")
+    qh, kh, vh, doh, oh = (_seq_to_heads(x, P, group, kernels) for x in (q, k, v, do, o))
+    lse_h = _lse_seq_to_heads(lse, P, group, kernels)
     dqh, dkh, dvh = kernels.ring_attn_bwd(qh, kh, vh, oh, lse_h, doh, 1, "contiguous", causal,
                                           softmax_scale=softmax_scale)
-    return to_seq(dqh), to_seq(dkh), to_seq(dvh)
+    return tuple(_heads_to_seq(g, P, group, kernels) for g in (dqh, dkh, dvh))
+
+
+# ------------------------------------------------------------------ USP hybrid
+def usp_groups(Pr: int, Pu: int):
+    """The two process groups of the calling rank in a Pr x Pu grid of the
+    default group's P = Pr * Pu ranks, rank R = g * Pu + u: its Ulysses group
+    (the Pu ranks of ring group g, in order of u) and its ring group (the Pr
+    ranks with the same u, in order of g).  Every rank must call this, in the
+    same order, because creating a group is collective."""
+    P = dist.get_world_size()
+    if Pr * Pu != P:
+        raise ValueError(f"Pr * Pu = {Pr * Pu} != world size {P}")
+    R = dist.get_rank()
+    mine_u = mine_r = None
+    for g in range(Pr):
+        grp = dist.new_group([g * Pu + u for u in range(Pu)])
+        if R // Pu == g:
+            mine_u = grp
+    for u in range(Pu):
+        grp = dist.new_group([g * Pu + u for g in range(Pr)])
+        if R % Pu == u:
+            mine_r = grp
+    return mine_u, mine_r
+
+
+def usp_attn_fwd_dist(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, layout: str = "contiguous",
+                      causal: bool = True, cu_seqlens: Optional[Sequence[int]] = None, groups=None,
+                      softmax_scale: float = 0.0, kernels=_api):
+    """The Ulysses-inside / Ring-across hybrid over a Pr x Pu rank grid
+    (compassingai, closing section; pwwt.cn §6).  ``groups`` = (Ulysses
+    group, ring group) from ``usp_groups``.  Rank (g, u) holds rows
+    [u*n, (u+1)*n) of ring shard g of ``layout`` over Pr (q [n, hq, dh], k, v
+    [n, hkv, dh]); Pu must divide hkv.  Steps: Ulysses seq->head inside the
+    group (the group's m = Pu*n rows of head block u), the ring over the Pr
+    groups for that head block, Ulysses head->seq.  Returns this rank's
+    (O [n, hq, dh] fp32, LSE [hq, n] fp32)."""
+    ug, rg = groups
+    Pu = dist.get_world_size(ug)
+    if k.shape[1] % Pu != 0:
+        raise ValueError(f"Pu = {Pu} must divide the KV head count {k.shape[1]}")
+    qh, kh, vh = (_seq_to_heads(x, Pu, ug, kernels) for x in (q, k, v))
+    o_h, lse_h = ring_attn_fwd_dist(qh, kh, vh, layout, causal, cu_seqlens, rg, softmax_scale, kernels)
+    return _heads_to_seq(o_h, Pu, ug, kernels), _lse_heads_to_seq(lse_h, Pu, ug, kernels)
+
+
+def usp_attn_bwd_dist(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse: torch.Tensor,
+                      do: torch.Tensor, layout: str = "contiguous", causal: bool = True,
+                      cu_seqlens: Optional[Sequence[int]] = None, groups=None, softmax_scale: float = 0.0,
+                      kernels=_api):
+    """Backward of ``usp_attn_fwd_dist``: Q, K, V, dO, O and LSE to head
+    layout inside the Ulysses group, the ring backward over the ring group
+    for this head block, dQ, dK, dV back.  Returns this rank's (dQ [n, hq, dh],
+    dK, dV [n, hkv, dh]) fp32."""
+    ug, rg = groups
+    Pu = dist.get_world_size(ug)
+    if k.shape[1] % Pu != 0:
+        raise ValueError(f"Pu = {Pu} must divide the KV head count {k.shape[1]}")
+    qh, kh, vh, doh, oh = (_seq_to_heads(x, Pu, ug, kernels) for x in (q, k, v, do, o))
+    lse_h = _lse_seq_to_heads(lse, Pu, ug, kernels)
+    grads = ring_attn_bwd_dist(qh, kh, vh, oh, lse_h, doh, layout, causal, cu_seqlens, rg, softmax_scale, kernels)
+    return tuple(_heads_to_seq(g, Pu, ug, kernels) for g in grads)

@@ -9,6 +9,7 @@ pair's backward and the LSE merge, a reshape for the head-block split, and
 the library's own host scheduler for the skip decisions.  Every rank's result
 must equal the oracle's attention (or its gradient) over the whole sequence
 for that rank's rows."""
+import datetime
 import os
 import socket
 import sys
@@ -97,110 +98,139 @@ class OracleKernels:
         return x.permute(1, 0, 2, 3).reshape(n, p_ * hg, dh).contiguous()
 
 
-def _worker(rank, world, port, kind, cfg, results):
+def _run_case(rank, world, kind, cfg):
+    """One case on this rank: the distributed entry point with the stand-ins."""
+    from context_exact_attention_step_b200 import distributed as D, synth
+    from oracle import ref
+    S, hq, hkv, dh = cfg["S"], cfg["hq"], cfg["hkv"], cfg["dh"]
+    q, k, v = (t.double() for t in synth.qkv(S, hq, hkv, dh))
+    layout = cfg.get("layout", "contiguous")
+    rows = _rows(S, world, kind, cfg, rank)
+    idx = torch.from_numpy(rows)
+    groups = D.usp_groups(cfg["Pr"], cfg["Pu"]) if kind.startswith("usp") else None
+    if kind == "usp":
+        o, lse = D.usp_attn_fwd_dist(q[idx], k[idx], v[idx], layout, cfg["causal"], cfg.get("cu"), groups,
+                                     kernels=OracleKernels)
+        return o.numpy(), lse.numpy()
+    if kind == "ring":
+        o, lse = D.ring_attn_fwd_dist(q[idx], k[idx], v[idx], layout, cfg["causal"], cfg.get("cu"),
+                                      kernels=OracleKernels)
+        return o.numpy(), lse.numpy()
+    if kind == "ulysses":
+        o, lse = D.ulysses_attn_fwd_dist(q[idx], k[idx], v[idx], cfg["causal"], kernels=OracleKernels)
+        return o.numpy(), lse.numpy()
+    # the backward: the forward's merged O and LSE of this rank's rows, from the oracle
+    do = synth.normal((S, hq, dh), synth.SEED_DO, 0.5).double()
+    o_all, lse_all = ref.attention(q.numpy(), k.numpy(), v.numpy(), causal=cfg["causal"], cu_seqlens=cfg.get("cu"))
+    o, lse = torch.from_numpy(o_all[rows]), torch.from_numpy(np.ascontiguousarray(lse_all[:, rows]))
+    if kind == "usp_bwd":
+        grads = D.usp_attn_bwd_dist(q[idx], k[idx], v[idx], o, lse, do[idx], layout, cfg["causal"], cfg.get("cu"),
+                                    groups, kernels=OracleKernels)
+    elif kind == "ring_bwd":
+        grads = D.ring_attn_bwd_dist(q[idx], k[idx], v[idx], o, lse, do[idx], layout, cfg["causal"], cfg.get("cu"),
+                                     kernels=OracleKernels)
+    else:
+        grads = D.ulysses_attn_bwd_dist(q[idx], k[idx], v[idx], o, lse, do[idx], cfg["causal"],
+                                        kernels=OracleKernels)
+    return tuple(g.numpy() for g in grads)
+
+
+def _worker(rank, world, port, cases, results):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
     sys.path.insert(0, ROOT)
-    dist.init_process_group("gloo", rank=rank, world_size=world)
+    # a short timeout: ranks that fall out of step end with an error, not a hang
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
     try:
-        from context_exact_attention_step_b200 import distributed as D, synth
-        from oracle import ref
-        S, hq, hkv, dh = cfg["S"], cfg["hq"], cfg["hkv"], cfg["dh"]
-        q, k, v = (t.double() for t in synth.qkv(S, hq, hkv, dh))
-        layout = cfg.get("layout", "contiguous")
-        rows = ref.shard_positions(S, world, layout, rank)
-        idx = torch.from_numpy(rows)
-        if kind == "ring":
-            o, lse = D.ring_attn_fwd_dist(q[idx], k[idx], v[idx], layout, cfg["causal"], cfg.get("cu"),
-                                          kernels=OracleKernels)
-            results[rank] = (o.numpy(), lse.numpy())
-        elif kind == "ulysses":
-            o, lse = D.ulysses_attn_fwd_dist(q[idx], k[idx], v[idx], cfg["causal"], kernels=OracleKernels)
-            results[rank] = (o.numpy(), lse.numpy())
-        else:
-            # the forward's merged O and LSE of this rank's rows, from the oracle
-            do = synth.normal((S, hq, dh), synth.SEED_DO, 0.5).double()
-            o_all, lse_all = ref.attention(q.numpy(), k.numpy(), v.numpy(), causal=cfg["causal"],
-                                           cu_seqlens=cfg.get("cu"))
-            o, lse = torch.from_numpy(o_all[rows]), torch.from_numpy(np.ascontiguousarray(lse_all[:, rows]))
-            if kind == "ring_bwd":
-                grads = D.ring_attn_bwd_dist(q[idx], k[idx], v[idx], o, lse, do[idx], layout, cfg["causal"],
-                                             cfg.get("cu"), kernels=OracleKernels)
-            else:
-                grads = D.ulysses_attn_bwd_dist(q[idx], k[idx], v[idx], o, lse, do[idx], cfg["causal"],
-                                                kernels=OracleKernels)
-            results[rank] = tuple(g.numpy() for g in grads)
+        for name, kind, cfg in cases:
+            results[(name, rank)] = _run_case(rank, world, kind, cfg)
     finally:
         dist.destroy_process_group()
 
 
-def _run(kind, world, cfg):
+def _rows(S, world, kind, cfg, r):
+    """Global positions of rank r's rows, in its storage order."""
+    from oracle import ref
+    layout = cfg.get("layout", "contiguous")
+    if kind.startswith("usp"):
+        Pr, Pu = cfg["Pr"], cfg["Pu"]
+        n = S // world
+        return ref.shard_positions(S, Pr, layout, r // Pu)[(r % Pu) * n:(r % Pu + 1) * n]
+    return ref.shard_positions(S, world, layout, r)
+
+
+# every case: (name, kind, world, cfg); the cases of one world size run in one
+# set of spawned ranks, one after another in the same process group
+CASES = []
+for _layout in ("contiguous", "zigzag", "striped"):
+    for _world in (2, 4):
+        CASES.append((f"ring-{_layout}-{_world}", "ring", _world,
+                      dict(S=64, hq=4, hkv=2, dh=8, layout=_layout, causal=True)))
+CASES += [
+    ("ring-zigzag-3", "ring", 3, dict(S=48, hq=2, hkv=1, dh=8, layout="zigzag", causal=True)),
+    ("ring-docs-noncausal-4", "ring", 4, dict(S=64, hq=2, hkv=2, dh=8, layout="zigzag", causal=False,
+                                              cu=[0, 5, 6, 40, 64])),
+    ("ring-docs-2", "ring", 2, dict(S=64, hq=2, hkv=2, dh=8, layout="contiguous", causal=True, cu=[0, 5, 6, 40, 64])),
+    ("ulysses-2", "ulysses", 2, dict(S=32, hq=8, hkv=4, dh=8, causal=True)),
+    ("ulysses-4", "ulysses", 4, dict(S=32, hq=8, hkv=4, dh=8, causal=True)),
+    ("ulysses-noncausal-2", "ulysses", 2, dict(S=32, hq=4, hkv=2, dh=8, causal=False)),
+    ("ring_bwd-contiguous-2", "ring_bwd", 2, dict(S=64, hq=4, hkv=2, dh=8, layout="contiguous", causal=True)),
+    ("ring_bwd-zigzag-4", "ring_bwd", 4, dict(S=64, hq=4, hkv=2, dh=8, layout="zigzag", causal=True)),
+    ("ring_bwd-striped-2", "ring_bwd", 2, dict(S=64, hq=4, hkv=2, dh=8, layout="striped", causal=True)),
+    ("ring_bwd-striped-4", "ring_bwd", 4, dict(S=64, hq=4, hkv=2, dh=8, layout="striped", causal=True)),
+    ("ring_bwd-docs-3", "ring_bwd", 3, dict(S=48, hq=2, hkv=1, dh=8, layout="zigzag", causal=True,
+                                            cu=[0, 7, 8, 30, 48])),
+    ("ring_bwd-noncausal-2", "ring_bwd", 2, dict(S=32, hq=2, hkv=2, dh=8, layout="contiguous", causal=False)),
+    ("ulysses_bwd-2", "ulysses_bwd", 2, dict(S=32, hq=8, hkv=4, dh=8, causal=True)),
+    ("ulysses_bwd-4", "ulysses_bwd", 4, dict(S=32, hq=8, hkv=4, dh=8, causal=True)),
+    ("ulysses_bwd-noncausal-2", "ulysses_bwd", 2, dict(S=32, hq=4, hkv=2, dh=8, causal=False)),
+]
+for _layout in ("contiguous", "zigzag", "striped"):
+    CASES.append((f"usp-{_layout}-2x2", "usp", 4,
+                  dict(S=64, hq=4, hkv=2, dh=8, layout=_layout, causal=True, Pr=2, Pu=2)))
+CASES += [
+    ("usp-docs-1x4", "usp", 4, dict(S=64, hq=8, hkv=4, dh=8, layout="zigzag", causal=True, Pr=1, Pu=4,
+                                    cu=[0, 9, 40, 64])),
+    ("usp-docs-noncausal-4x1", "usp", 4, dict(S=64, hq=4, hkv=4, dh=8, layout="zigzag", causal=False, Pr=4, Pu=1,
+                                              cu=[0, 9, 40, 64])),
+    ("usp_bwd-zigzag-2x2", "usp_bwd", 4, dict(S=64, hq=4, hkv=2, dh=8, layout="zigzag", causal=True, Pr=2, Pu=2)),
+    ("usp_bwd-striped-2x2", "usp_bwd", 4, dict(S=64, hq=4, hkv=2, dh=8, layout="striped", causal=True, Pr=2, Pu=2)),
+    ("usp_bwd-docs-2x2", "usp_bwd", 4, dict(S=64, hq=4, hkv=2, dh=8, layout="contiguous", causal=True, Pr=2, Pu=2,
+                                            cu=[0, 5, 6, 40, 64])),
+]
+_RESULTS = {}
+
+
+def _results(world):
+    if world not in _RESULTS:
+        cases = [(name, kind, cfg) for name, kind, w, cfg in CASES if w == world]
+        manager = mp.Manager()
+        results = manager.dict()
+        mp.spawn(_worker, args=(world, _free_port(), cases, results), nprocs=world, join=True)
+        _RESULTS[world] = dict(results)
+    return _RESULTS[world]
+
+
+@pytest.mark.parametrize("name", [c[0] for c in CASES])
+def test_distributed_case(name):
+    """Every rank's rows equal the oracle's attention (or its gradient) over
+    the whole sequence."""
     from oracle import ref
     from context_exact_attention_step_b200 import synth
-    manager = mp.Manager()
-    results = manager.dict()
-    mp.spawn(_worker, args=(world, _free_port(), kind, cfg, results), nprocs=world, join=True)
+    _, kind, world, cfg = next(c for c in CASES if c[0] == name)
+    results = _results(world)
     S, hq, hkv, dh = cfg["S"], cfg["hq"], cfg["hkv"], cfg["dh"]
     q, k, v = (t.double().numpy() for t in synth.qkv(S, hq, hkv, dh))
     if kind.endswith("_bwd"):
         do = synth.normal((S, hq, dh), synth.SEED_DO, 0.5).double().numpy()
         want = ref.attention_bwd(q, k, v, do, causal=cfg["causal"], cu_seqlens=cfg.get("cu"))
         for r in range(world):
-            rows = ref.shard_positions(S, world, cfg.get("layout", "contiguous"), r)
-            for got, w, what in zip(results[r], want, ("dQ", "dK", "dV")):
+            rows = _rows(S, world, kind, cfg, r)
+            for got, w, what in zip(results[(name, r)], want, ("dQ", "dK", "dV")):
                 np.testing.assert_allclose(got, w[rows], atol=1e-10, err_msg=f"{what} of rank {r}")
         return
     want_o, want_l = ref.attention(q, k, v, causal=cfg["causal"], cu_seqlens=cfg.get("cu"))
     for r in range(world):
-        rows = ref.shard_positions(S, world, cfg.get("layout", "contiguous"), r)
-        o, lse = results[r]
+        rows = _rows(S, world, kind, cfg, r)
+        o, lse = results[(name, r)]
         np.testing.assert_allclose(o, want_o[rows], atol=1e-10)
         np.testing.assert_allclose(lse, want_l[:, rows], atol=1e-10)
-
-
-@pytest.mark.parametrize("layout", ["contiguous", "zigzag", "striped"])
-@pytest.mark.parametrize("world", [2, 4])
-def test_ring_over_ranks(layout, world):
-    _run("ring", world, dict(S=64, hq=4, hkv=2, dh=8, layout=layout, causal=True))
-
-
-def test_ring_over_three_ranks():
-    # an odd ring: every rank's shard visits the others in the same order
-    _run("ring", 3, dict(S=48, hq=2, hkv=1, dh=8, layout="zigzag", causal=True))
-
-
-def test_ring_over_ranks_noncausal_documents():
-    _run("ring", 4, dict(S=64, hq=2, hkv=2, dh=8, layout="zigzag", causal=False, cu=[0, 5, 6, 40, 64]))
-    _run("ring", 2, dict(S=64, hq=2, hkv=2, dh=8, layout="contiguous", causal=True, cu=[0, 5, 6, 40, 64]))
-
-
-@pytest.mark.parametrize("world", [2, 4])
-def test_ulysses_over_ranks(world):
-    _run("ulysses", world, dict(S=32, hq=8, hkv=4, dh=8, causal=True))
-
-
-def test_ulysses_over_ranks_noncausal():
-    _run("ulysses", 2, dict(S=32, hq=4, hkv=2, dh=8, causal=False))
-
-
-@pytest.mark.parametrize("layout,world", [("contiguous", 2), ("zigzag", 4), ("striped", 2), ("striped", 4)])
-def test_ring_bwd_over_ranks(layout, world):
-    _run("ring_bwd", world, dict(S=64, hq=4, hkv=2, dh=8, layout=layout, causal=True))
-
-
-def test_ring_bwd_over_three_ranks_documents():
-    # an odd ring with documents: some steps are skipped, yet every shard's
-    # gradient still makes the full circle home
-    _run("ring_bwd", 3, dict(S=48, hq=2, hkv=1, dh=8, layout="zigzag", causal=True, cu=[0, 7, 8, 30, 48]))
-
-
-def test_ring_bwd_over_ranks_noncausal():
-    _run("ring_bwd", 2, dict(S=32, hq=2, hkv=2, dh=8, layout="contiguous", causal=False))
-
-
-@pytest.mark.parametrize("world", [2, 4])
-def test_ulysses_bwd_over_ranks(world):
-    _run("ulysses_bwd", world, dict(S=32, hq=8, hkv=4, dh=8, causal=True))
-
-
-def test_ulysses_bwd_over_ranks_noncausal():
-    _run("ulysses_bwd", 2, dict(S=32, hq=4, hkv=2, dh=8, causal=False))

@@ -70,3 +70,20 @@ def test_ulysses_bwd_dist_one_rank(one_rank_group):
     want = ref.attention_bwd(f64(q), f64(k), f64(v), f64(do), causal=False)
     for got, w, what in zip((dq, dk, dv), want, ("dQ", "dK", "dV")):
         check_grad(got, w, f"ulysses backward over one rank: {what}")
+
+
+def test_usp_dist_one_rank(one_rank_group):
+    # the hybrid's two process groups on a 1 x 1 grid: forward and backward
+    S, hq, hkv, dh = 768, 4, 2, 64
+    q, k, v = synth.qkv(S, hq, hkv, dh)
+    do = synth.normal((S, hq, dh), synth.SEED_DO, 0.5)
+    qd, kd, vd, dod = (t.cuda() for t in (q, k, v, do))
+    groups = D.usp_groups(1, 1)
+    o, lse = D.usp_attn_fwd_dist(qd, kd, vd, "zigzag", True, None, groups)
+    dq, dk, dv = D.usp_attn_bwd_dist(qd, kd, vd, o, lse, dod, "zigzag", True, None, groups)
+    torch.cuda.synchronize()
+    want_o, want_l = ref.attention(f64(q), f64(k), f64(v), causal=True)
+    compare(o, lse, want_o, want_l, what="usp over one rank")
+    want = ref.attention_bwd(f64(q), f64(k), f64(v), f64(do), causal=True)
+    for got, w, what in zip((dq, dk, dv), want, ("dQ", "dK", "dV")):
+        check_grad(got, w, f"usp backward over one rank: {what}")

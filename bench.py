@@ -403,6 +403,105 @@ def time_permute(reps=20):
     return dict(gbs=nbytes / (ms * 1e-3) / 1e9, ms=ms, bytes=nbytes)
 
 
+# ----------------------------------------------------------------- multi-GPU ring, rank by rank
+NVLINK_PEER_GBS = 770.0  # measured peer-copy bandwidth per direction on this hardware (B200, NVLink 5)
+
+
+def time_per_rank(w, reps=5):
+    """The kernel work of every rank of the multi-GPU ring (``distributed``),
+    run rank after rank on this GPU through the same entry points: forward,
+    the block pairs of the rank's live ring steps and its merge; backward, the
+    prep and, per live step, the dK/dV and dQ block-pair kernels.  The
+    exchanges cannot run on one GPU; their bytes per step and their time at
+    the peer-copy bandwidth are reported beside the compute."""
+    from context_exact_attention_step_b200 import api
+    from context_exact_attention_step_b200 import distributed as D
+    S, P, layout, cu = w["S"], w["P"], w["layout"], w["cu"]
+    if layout not in ("contiguous", "zigzag", "striped"):
+        raise SystemExit("--per-rank needs a ring workload")
+    hq, hkv, dh = w["hq"], w["hkv"], w["dh"]
+    n = S // P
+    dev = torch.device("cuda")
+    bwd = w.get("pass") == "bwd"
+    cu_dev = torch.tensor(cu, dtype=torch.int32, device=dev) if cu is not None else None
+    sch = api.ring_schedule(S, P, layout, True, cu)
+    if bwd:
+        qs, ks, vs, o, lse, dos = w["in"]
+    else:
+        qs, ks, vs = w["in"]
+        if w["dtype"] != torch.bfloat16:
+            raise SystemExit("--per-rank takes bf16 workloads")
+        if layout != "contiguous":
+            reorder = api.zigzag_reorder if layout == "zigzag" else api.striped_reorder
+            qs, ks, vs = (reorder(t, P) for t in (qs, ks, vs))
+    parts_o = [torch.empty((n, hq, dh), device=dev, dtype=torch.float32) for _ in range(P)]
+    parts_l = [torch.empty((hq, n), device=dev, dtype=torch.float32) for _ in range(P)]
+    o_r = torch.empty((n, hq, dh), device=dev, dtype=torch.float32)
+    l_r = torch.empty((hq, n), device=dev, dtype=torch.float32)
+    lg = torch.empty((hq, n), device=dev, dtype=torch.float32)
+    dd = torch.empty_like(lg)
+    dq = torch.empty((n, hq, dh), device=dev, dtype=torch.float32)
+    dk = torch.empty((n, hkv, dh), device=dev, dtype=torch.float32)
+    dv = torch.empty_like(dk)
+    rows = lambda t, r: t[r * n:(r + 1) * n]
+    lse_r = [lse[:, r * n:(r + 1) * n].contiguous() for r in range(P)] if bwd else None
+
+    def rank_work(r):
+        qc = D.query_chunks(S, P, layout, r)
+        if bwd:
+            api.attn_bwd_prep(rows(o, r), lse_r[r], rows(dos, r), lg=lg, dd=dd)
+        used = 0
+        for t in range(P):
+            if not sch["launched"][r * P + t]:
+                continue
+            j = (r - t) % P
+            kc = D.key_chunks(S, P, layout, r, j)
+            if bwd:
+                api.block_attn_bwd(rows(qs, r), rows(ks, j), rows(vs, j), rows(dos, r), lg, dd, qc, kc, True, cu_dev,
+                                   dk=dk, dv=dv, parts=2, accumulate=t > 0)
+                api.block_attn_bwd(rows(qs, r), rows(ks, j), rows(vs, j), rows(dos, r), lg, dd, qc, kc, True, cu_dev,
+                                   dq=dq, parts=1, accumulate=t > 0)
+            else:
+                api.block_attn_fwd(rows(qs, r), rows(ks, j), rows(vs, j), qc, kc, True, cu_dev,
+                                   o=parts_o[used], lse=parts_l[used])
+            used += 1
+        if not bwd:
+            api.lse_merge(parts_o[:used], parts_l[:used], o_out=o_r, lse_out=l_r)
+
+    for r in range(P):  # warm-up
+        rank_work(r)
+    torch.cuda.synchronize()
+    ms = []
+    for r in range(P):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            rank_work(r)
+        b.record()
+        torch.cuda.synchronize()
+        ms.append(a.elapsed_time(b) / reps)
+    if api.device_error():
+        raise RuntimeError("device error word set during the per-rank runs")
+    unit = (10.0 if bwd else 4.0) * dh * hq
+    pairs = [int(sum(sch["live_pairs"][r * P + t] for t in range(P))) for r in range(P)]
+    busiest = int(np.argmax(ms))
+    kv_bytes = 2 * n * hkv * dh * 2
+    grad_bytes = 2 * n * hkv * dh * 4 if bwd else 0
+    live_steps = [int(sum(sch["launched"][r * P + t] for t in range(P))) for r in range(P)]
+    return {
+        "what": ("backward: prep, then per live ring step the dK/dV and dQ block-pair kernels" if bwd else
+                 "forward: the block pairs of the rank's live ring steps, then its merge")
+                + "; ranks run one after another on this GPU, exchanges not included",
+        "ms": ms, "max_ms": max(ms), "live_steps": live_steps,
+        "tflops_busiest_rank": unit * pairs[busiest] / (ms[busiest] * 1e-3) / 1e12,
+        "tflops_P_gpus": w["flops"] / (max(ms) * 1e-3) / 1e12,
+        "exchange_bytes_per_step": kv_bytes + grad_bytes,
+        "exchange_ms_per_step_at_peer_bw": (kv_bytes + grad_bytes) / (NVLINK_PEER_GBS * 1e9) * 1e3,
+        "compute_ms_per_live_step_busiest": ms[busiest] / max(1, live_steps[busiest]),
+        "peer_bw_gbs": NVLINK_PEER_GBS,
+    }
+
+
 # ----------------------------------------------------------------- CPU oracle
 def oracle_sample_rate(w, target_s=12.0, max_rows=1024, seed=0, bwd=False):
     """Times the fp64 oracle on a bounded sample of the same workload: batches
@@ -548,6 +647,8 @@ def run_ours(args, ws, rank, local):
     if perm:
         line["a2a_permute"] = {"gbs": perm["gbs"], "frac_hbm": perm["gbs"] / pk["hbm_gbs"], "ms": perm["ms"],
                                "bytes": perm["bytes"], "workload": "ulysses_gqa_128k Q,K,V seq->head + fp32 O head->seq"}
+    if args.per_rank:
+        line["per_rank"] = time_per_rank(w)
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_sample_rate(w, bwd=bwd)
     if rank == 0:
@@ -580,6 +681,8 @@ def main():
     ap.add_argument("--pass", dest="pass_", default="fwd", choices=["fwd", "bwd"],
                     help="bwd: time the ring backward (dQ, dK, dV) of a ring workload instead of the forward")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--per-rank", action="store_true",
+                    help="also time each rank's kernel work of the multi-GPU ring (ring workloads)")
     ap.add_argument("--seq-len", type=int, default=None,
                     help="override the workload's sequence length (smaller cases for profiler captures)")
     args = ap.parse_args()

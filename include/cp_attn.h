@@ -39,7 +39,7 @@ extern "C" {
 typedef enum {
   CP_OK = 0,
   CP_ERR_INVALID_ARG = 1,  /* a size, count or pointer is out of range       */
-  CP_ERR_UNSUPPORTED = 2,  /* valid request outside what this build supports  */
+  CP_ERR_UNSUPPORTED = 2,  /* valid request outside what the library supports */
   CP_ERR_ALIGNMENT = 3,    /* a device pointer is not 16-byte aligned        */
   CP_ERR_WORKSPACE = 4,    /* workspace missing or smaller than required      */
   CP_ERR_CUDA = 5          /* the CUDA runtime reported an error              */

@@ -558,29 +558,46 @@ def run_reference(args, ws, rank):
         cu = synth.cu_seqlens_from_lengths(synth.doc_lengths(S, cfg["doc_lo"], cfg["doc_hi"])).tolist()
     rng = np.random.default_rng(1)
     rows_per_step = 32
+    bwd = args.pass_ == "bwd"
+    if bwd:
+        do = synth.normal((S, hq, dh), synth.SEED_DO, 0.5).double().numpy()
 
     def step():
         rows = np.sort(rng.integers(0, S, rows_per_step))
-        ref.attention(q[rows], k, v, causal=True, cu_seqlens=cu, qpos=rows)
+        if bwd:  # the gradient work of these query rows (their dQ, their share of dK, dV)
+            ref.attention_bwd(q[rows], k, v, do[rows], causal=True, cu_seqlens=cu, qpos=rows)
+        else:
+            ref.attention(q[rows], k, v, causal=True, cu_seqlens=cu, qpos=rows)
         if cu is None:
             return float((rows + 1).sum())
         starts = np.asarray(cu)[np.searchsorted(cu, rows, side="right") - 1]
         return float((rows - starts + 1).sum())
 
+    # the workload's identity, as the GPU arm reports it (causal pairs in
+    # closed form: S(S+1)/2, or the sum of L(L+1)/2 over the documents)
+    lens = np.diff(np.asarray(cu, dtype=np.int64)) if cu is not None else np.array([S], dtype=np.int64)
+    pairs = int((lens * (lens + 1) // 2).sum())
+    ref_config = {"workload": name, **{k_: cfg[k_] for k_ in ("S", "hq", "hkv", "dh", "P", "layout")},
+                  "causal": True, "input_dtype": cfg["dtype"], "admitted_pairs": pairs,
+                  "flops_per_step": (10.0 if bwd else 4.0) * dh * hq * pairs,
+                  **({k_: cfg[k_] for k_ in ("Pr", "Pu", "ring_layout")} if cfg["layout"] == "usp" else {})}
+    if bwd:
+        ref_config["pass"] = "backward: the gradient of the sampled query rows"
     for _ in range(args.warmup):
         step()
     t0 = time.perf_counter()
     live = sum(step() for _ in range(args.steps))
     dt = time.perf_counter() - t0
-    val = 4.0 * dh * hq * live / dt / 1e12
+    val = (10.0 if bwd else 4.0) * dh * hq * live / dt / 1e12
     cores = len(os.sched_getaffinity(0))
     line = {
-        "impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": ws,
+        "impl": "reference", "metric": METRIC_BWD if bwd else METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": name, **{k_: cfg[k_] for k_ in ("S", "hq", "hkv", "dh", "P", "layout")}},
+        "config": ref_config,
         "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                         "sample": f"{rows_per_step} seeded query rows x all keys x all heads per step"},
+                         "sample": f"{'gradient of ' if bwd else ''}{rows_per_step} seeded query rows x all keys x "
+                                   f"all heads per step"},
         "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)

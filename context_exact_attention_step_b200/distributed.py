@@ -132,7 +132,7 @@ def _heads_to_seq(x_h: torch.Tensor, P: int, group, kernels) -> torch.Tensor:
     """Inverse of _seq_to_heads: [P*n, hb, dh] -> [n, P*hb, dh]."""
     rows, hb, dh = x_h.shape
     n = rows // P
-    blocks = torch.empty_like(x_h).view(P, n, hb, dh)
+    blocks = torch.empty((P, n, hb, dh), dtype=x_h.dtype, device=x_h.device)
     dist.all_to_all_single(blocks, x_h.view(P, n, hb, dh).contiguous(), group=group)
     return kernels.head_block_split(blocks, P, inverse=True)
 
@@ -142,7 +142,7 @@ def _lse_seq_to_heads(lse: torch.Tensor, P: int, group, kernels) -> torch.Tensor
     block p goes to rank p, and the [P][h/P][n] slabs received become
     [h/P][P][n]."""
     h, n = lse.shape
-    got = torch.empty_like(lse)
+    got = torch.empty((h, n), dtype=lse.dtype, device=lse.device)
     dist.all_to_all_single(got, lse.contiguous(), group=group)
     return kernels.head_block_split(got.view(P, h // P, 1, n), P, inverse=True).view(h // P, P * n)
 

@@ -123,6 +123,8 @@ def _run_case(rank, world, kind, cfg):
     do = synth.normal((S, hq, dh), synth.SEED_DO, 0.5).double()
     o_all, lse_all = ref.attention(q.numpy(), k.numpy(), v.numpy(), causal=cfg["causal"], cu_seqlens=cfg.get("cu"))
     o, lse = torch.from_numpy(o_all[rows]), torch.from_numpy(np.ascontiguousarray(lse_all[:, rows]))
+    if cfg.get("lse_transposed"):  # same values, column-major storage
+        lse = lse.T.contiguous().T
     if kind == "usp_bwd":
         grads = D.usp_attn_bwd_dist(q[idx], k[idx], v[idx], o, lse, do[idx], layout, cfg["causal"], cfg.get("cu"),
                                     groups, kernels=OracleKernels)
@@ -183,6 +185,8 @@ CASES += [
     ("ulysses_bwd-2", "ulysses_bwd", 2, dict(S=32, hq=8, hkv=4, dh=8, causal=True)),
     ("ulysses_bwd-4", "ulysses_bwd", 4, dict(S=32, hq=8, hkv=4, dh=8, causal=True)),
     ("ulysses_bwd-noncausal-2", "ulysses_bwd", 2, dict(S=32, hq=4, hkv=2, dh=8, causal=False)),
+    ("ulysses_bwd-lse-transposed-2", "ulysses_bwd", 2, dict(S=32, hq=4, hkv=2, dh=8, causal=True,
+                                                            lse_transposed=True)),
 ]
 for _layout in ("contiguous", "zigzag", "striped"):
     CASES.append((f"usp-{_layout}-2x2", "usp", 4,

@@ -458,9 +458,9 @@ def time_per_rank(w, reps=5):
             kc = D.key_chunks(S, P, layout, r, j)
             if bwd:
                 api.block_attn_bwd(rows(qs, r), rows(ks, j), rows(vs, j), rows(dos, r), lg, dd, qc, kc, True, cu_dev,
-                                   dk=dk, dv=dv, parts=2, accumulate=t > 0)
+                                   dk=dk, dv=dv, parts=api.BWD_DKDV, accumulate=t > 0)
                 api.block_attn_bwd(rows(qs, r), rows(ks, j), rows(vs, j), rows(dos, r), lg, dd, qc, kc, True, cu_dev,
-                                   dq=dq, parts=1, accumulate=t > 0)
+                                   dq=dq, parts=api.BWD_DQ, accumulate=t > 0)
             else:
                 api.block_attn_fwd(rows(qs, r), rows(ks, j), rows(vs, j), qc, kc, True, cu_dev,
                                    o=parts_o[used], lse=parts_l[used])

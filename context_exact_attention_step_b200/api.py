@@ -347,6 +347,10 @@ def ring_attn_bwd(q, k, v, o, lse, do, P, layout="contiguous", causal=True, cu_s
     return dq, dk, dv
 
 
+BWD_DQ = _lib.CP_BWD_DQ      # block_attn_bwd parts: the dQ kernel
+BWD_DKDV = _lib.CP_BWD_DKDV  # the dK/dV kernel
+
+
 def attn_bwd_prep(o, lse, do, lg=None, dd=None, stream=None):
     """Per-row vectors of the backward: lg = LSE * log2(e) (0 where LSE is
     -inf) and dd = rowsum(dO * O), both [hq, n] fp32, from the forward's o
@@ -364,10 +368,11 @@ def attn_bwd_prep(o, lse, do, lg=None, dd=None, stream=None):
 
 
 def block_attn_bwd(q, k, v, do, lg, dd, q_chunks=None, k_chunks=None, causal=True, cu_seqlens=None,
-                   softmax_scale=0.0, dq=None, dk=None, dv=None, parts=3, accumulate=False, stream=None):
+                   softmax_scale=0.0, dq=None, dk=None, dv=None, parts=BWD_DQ | BWD_DKDV, accumulate=False,
+                   stream=None):
     """Gradient contribution of one block pair: q, do [n_q, hq, dh] vs k, v
     [n_k, hkv, dh] (bf16, CUDA), lg, dd from ``attn_bwd_prep`` of the query
-    rows; chunks and mask as ``block_attn_fwd``.  parts: 1 dQ, 2 dK/dV, 3
+    rows; chunks and mask as ``block_attn_fwd``.  parts: BWD_DQ, BWD_DKDV or
     both.  accumulate: add to dq / dk / dv instead of overwriting them.
     Returns (dq [n_q, hq, dh], dk, dv [n_k, hkv, dh]) fp32 (None for a part
     not computed and not given)."""

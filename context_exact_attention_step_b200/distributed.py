@@ -215,7 +215,7 @@ def ring_attn_bwd_dist(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: tor
         k_chunks = key_chunks(S, P, layout, r, j)
         if live:
             kernels.block_attn_bwd(q, kv[:n], kv[n:], do, lg, dd, q_chunks, k_chunks, causal, cu_dev, softmax_scale,
-                                   dk=dkv[:n], dv=dkv[n:], parts=2, accumulate=t > 0)
+                                   dk=dkv[:n], dv=dkv[n:], parts=_api.BWD_DKDV, accumulate=t > 0)
         elif t == 0:
             dkv.zero_()
         # the shard's gradient moves on with it; the last move brings it home
@@ -225,7 +225,7 @@ def ring_attn_bwd_dist(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: tor
                                             dist.P2POp(dist.irecv, dkv_next, recv_from, group)])
         if live:
             kernels.block_attn_bwd(q, kv[:n], kv[n:], do, lg, dd, q_chunks, k_chunks, causal, cu_dev, softmax_scale,
-                                   dq=dq, parts=1, accumulate=t > 0)
+                                   dq=dq, parts=_api.BWD_DQ, accumulate=t > 0)
         elif t == 0:
             dq.zero_()
         for req in reqs:

@@ -63,13 +63,14 @@ class OracleKernels:
     @staticmethod
     def block_attn_bwd(q, k, v, do, lg, dd, q_chunks, k_chunks, causal, cu_dev, scale, dq=None, dk=None, dv=None,
                        parts=3, accumulate=False):
+        from context_exact_attention_step_b200 import api
         from oracle import ref
         qpos = np.concatenate([np.arange(a, a + n) for a, n in q_chunks])
         kpos = np.concatenate([np.arange(a, a + n) for a, n in k_chunks])
         cu = None if cu_dev is None else cu_dev.tolist()
         grads = ref.ring_pair_bwd(q.numpy(), k.numpy(), v.numpy(), do.numpy(), None, lg.numpy(), qpos, kpos, causal,
                                   cu, scale or None, d_r=dd.numpy())
-        for g, out, bit in zip(grads, (dq, dk, dv), (1, 2, 2)):
+        for g, out, bit in zip(grads, (dq, dk, dv), (api.BWD_DQ, api.BWD_DKDV, api.BWD_DKDV)):
             if parts & bit:
                 t = torch.from_numpy(g).to(out.dtype)
                 if accumulate:

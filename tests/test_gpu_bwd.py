@@ -257,10 +257,10 @@ def test_block_bwd_parts_and_accumulate():
     base_k = torch.randn(S, hkv, dh, device="cuda")
     dq = base_q.clone()
     dk, dv = base_k.clone(), base_k.clone()
-    api.block_attn_bwd(qd, kd, vd, dod, lg, dd, causal=False, dq=dq, parts=1, accumulate=True)
+    api.block_attn_bwd(qd, kd, vd, dod, lg, dd, causal=False, dq=dq, parts=api.BWD_DQ, accumulate=True)
     torch.cuda.synchronize()
-    assert torch.equal(dk, base_k) and torch.equal(dv, base_k), "parts=1 must leave dK, dV alone"
-    api.block_attn_bwd(qd, kd, vd, dod, lg, dd, causal=False, dk=dk, dv=dv, parts=2, accumulate=True)
+    assert torch.equal(dk, base_k) and torch.equal(dv, base_k), "the dQ part alone must leave dK, dV alone"
+    api.block_attn_bwd(qd, kd, vd, dod, lg, dd, causal=False, dk=dk, dv=dv, parts=api.BWD_DKDV, accumulate=True)
     torch.cuda.synchronize()
     assert api.device_error() == 0
     wq, wk, wv = ref.attention_bwd(f64(q), f64(k), f64(v), f64(do), causal=False)

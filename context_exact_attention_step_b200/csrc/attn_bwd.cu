@@ -228,10 +228,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  const int h = blockIdx.x % plan.hq;
+  // Head-major: consecutive CTAs take the items of one head (heaviest first),
+  // so the CTAs running together stream the same head's K and V through L2.
+  const int h = blockIdx.x / plan.n_items;
   const int hk = h / (plan.hq / plan.hkv);
   Own own;
-  decode_own(plan, plan.items[blockIdx.x / plan.hq], own);
+  decode_own(plan, plan.items[blockIdx.x % plan.n_items], own);
   auto col_d = [](int) { return C::kColD; };
 
   // Registers: launched at 168 per thread (384 threads); inside its own
@@ -657,9 +659,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  const int hk = blockIdx.x % plan.hkv;
+  // Head-major, as in the dQ kernel: the CTAs running together share the
+  // query heads whose Q and dO tiles they stream.
+  const int hk = blockIdx.x / plan.n_items;
   Own own;
-  decode_own(plan, plan.items[blockIdx.x / plan.hkv], own);
+  decode_own(plan, plan.items[blockIdx.x % plan.n_items], own);
   auto col_r = [](int i) { return (i & 1) ? 128u : 0u; };
   auto stage_q = [&](int s) { return sStage + s * C::kStageBytes; };
   auto stage_do = [&](int s) { return sStage + s * C::kStageBytes + T::kTileBytes; };

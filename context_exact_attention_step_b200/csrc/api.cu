@@ -1,6 +1,7 @@
 // C ABI of the library (see include/cp_attn.h): argument validation, TMA
-// tensor maps, the ring / Ulysses composites and the host-only schedule
-// queries.  Host code only; the kernels live in attn_fwd.cu, merge.cu and
+// tensor maps, the ring / Ulysses / hybrid composites forward and backward,
+// the block-pair entry points and the host-only schedule queries.  Host code
+// only; the kernels live in attn_fwd.cu, attn_bwd.cu, merge.cu and
 // permute.cu.
 #include <cuda.h>
 #include <cudaTypedefs.h>

@@ -1,8 +1,11 @@
 /*
  * cp_attn.h -- C ABI of the B200 (sm_100a) context-parallel exact attention
  * library: ring-step block attention producing partial (O, LSE), the fp32 LSE
- * merge, the zigzag reorder and the Ulysses sequence<->head transpose, with
- * the P ranks of a context-parallel group held as virtual ranks on one GPU.
+ * merge, the zigzag and striped reorders, the Ulysses sequence<->head
+ * transpose and head-block split, the ring / Ulysses / hybrid (USP)
+ * composites with the P ranks of a context-parallel group held as virtual
+ * ranks on one GPU, their backward, and the backward of one block pair (the
+ * per-GPU step of a ring that spans GPUs).
  *
  * Conventions shared by every call
  * --------------------------------

@@ -143,10 +143,24 @@ def _worker(rank, world, port, cases, results):
     sys.path.insert(0, ROOT)
     # a short timeout: ranks that fall out of step end with an error, not a hang
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    # log every point-to-point exchange the distributed code posts:
+    # (op, peer, elements) per batch, in posting order
+    from context_exact_attention_step_b200 import distributed as D
+    post = D.dist.batch_isend_irecv
+    log = []
+
+    def logged(ops):
+        log.append(tuple(("send" if op.op is dist.isend else "recv", op.peer, op.tensor.numel()) for op in ops))
+        return post(ops)
+
+    D.dist.batch_isend_irecv = logged
     try:
         for name, kind, cfg in cases:
+            log.clear()
             results[(name, rank)] = _run_case(rank, world, kind, cfg)
+            results[("exchanges", name, rank)] = list(log)
     finally:
+        D.dist.batch_isend_irecv = post
         dist.destroy_process_group()
 
 
@@ -239,3 +253,23 @@ def test_distributed_case(name):
         o, lse = results[(name, r)]
         np.testing.assert_allclose(o, want_o[rows], atol=1e-10)
         np.testing.assert_allclose(lse, want_l[:, rows], atol=1e-10)
+
+
+@pytest.mark.parametrize("name", ["ring_bwd-docs-3", "ring_bwd-zigzag-4", "ring-docs-noncausal-4", "ring-zigzag-3"])
+def test_ring_exchanges_are_the_same_on_every_rank(name):
+    """Every rank posts the same exchanges in the same order, skipped steps
+    included: the ring forward moves K/V P - 1 times; the backward also moves
+    the shard's dK/dV P times (the last move brings it home).  Each batch sends
+    to rank r + 1 and receives from rank r - 1."""
+    _, kind, world, cfg = next(c for c in CASES if c[0] == name)
+    results = _results(world)
+    n = cfg["S"] // world
+    kv = 2 * n * cfg["hkv"] * cfg["dh"]
+    logs = [results[("exchanges", name, r)] for r in range(world)]
+    want = [kv] * (world - 1)
+    if kind == "ring_bwd":  # per step: K/V (except the last step), then dK/dV
+        want = [x for t in range(world) for x in ([kv] if t < world - 1 else []) + [kv]]
+    for r, log in enumerate(logs):
+        assert [batch[0][2] for batch in log] == want, f"rank {r}: {log}"
+        for batch in log:
+            assert batch == (("send", (r + 1) % world, batch[0][2]), ("recv", (r - 1) % world, batch[0][2]))

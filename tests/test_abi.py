@@ -197,7 +197,7 @@ def test_permute_and_merge_reject_bad_arguments():
 
 # ------------------------------------------------------------ scheduler
 @pytest.mark.parametrize("layout", ["contiguous", "zigzag", "striped"])
-@pytest.mark.parametrize("P", [1, 2, 4, 8])
+@pytest.mark.parametrize("P", [1, 2, 3, 4, 8, 16])
 @pytest.mark.parametrize("causal", [True, False])
 def test_schedule_matches_bruteforce(layout, P, causal):
     S = 16 * P * 2
@@ -212,19 +212,21 @@ def test_schedule_matches_bruteforce(layout, P, causal):
             assert sch["launched"][i] == (1 if live > 0 else 0)
 
 
-def test_schedule_varlen_matches_bruteforce():
-    S, P = 256, 4
-    cu = [0, 3, 70, 71, 200, 256]
-    sch = api.ring_schedule(S, P, "zigzag", True, cu)
-    cls = ref.pair_classes(S, P, "zigzag", True, cu)
+@pytest.mark.parametrize("layout,P,causal", [("zigzag", 4, True), ("contiguous", 4, True), ("zigzag", 16, True),
+                                             ("zigzag", 4, False), ("contiguous", 8, False)])
+def test_schedule_varlen_matches_bruteforce(layout, P, causal):
+    S = 256 * (2 if P == 16 else 1)
+    cu = [0, 3, 70, 71, 200, S]
+    sch = api.ring_schedule(S, P, layout, causal, cu)
+    cls = ref.pair_classes(S, P, layout, causal, cu)
     for (r, t), (j, live, _) in cls.items():
         assert sch["live_pairs"][r * P + t] == live
         assert sch["launched"][r * P + t] == (1 if live else 0)
         if live:
             # every query row that admits a key of the pair is computed
-            qp = ref.shard_positions(S, P, "zigzag", r)
-            kp = ref.shard_positions(S, P, "zigzag", j)
-            rows_live = ref.explicit_mask(qp, kp, True, cu).any(axis=1).sum()
+            qp = ref.shard_positions(S, P, layout, r)
+            kp = ref.shard_positions(S, P, layout, j)
+            rows_live = ref.explicit_mask(qp, kp, causal, cu).any(axis=1).sum()
             assert sch["q_rows"][r * P + t] >= rows_live
 
 

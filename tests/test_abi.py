@@ -7,6 +7,7 @@ import re
 
 import numpy as np
 import pytest
+from hypothesis import given, settings, strategies as st
 
 from context_exact_attention_step_b200 import _lib, api
 from context_exact_attention_step_b200._lib import cp_chunk, lib
@@ -246,3 +247,25 @@ def test_live_pair_count_against_oracle():
     assert api.count_live_pairs(64, True) == 64 * 65 // 2
     assert api.count_live_pairs(64, False) == 64 * 64
     assert api.count_live_pairs(131072, True) == 131072 * 131073 // 2
+
+
+@settings(max_examples=60, deadline=None)
+@given(st.data())
+def test_schedule_random_problems_match_bruteforce(data):
+    # random shard counts, layouts, masks and document tables: the host
+    # scheduler's source shard, admitted-pair count and launch decision of
+    # every (rank, step) equal the brute-force mask's
+    layout = data.draw(st.sampled_from(["contiguous", "zigzag", "striped"]))
+    P = data.draw(st.integers(1, 9))
+    unit = 2 * P if layout == "zigzag" else P
+    S = unit * data.draw(st.integers(1, max(1, 160 // unit)))
+    causal = data.draw(st.booleans())
+    cu = None
+    if layout != "striped" and S > 1 and data.draw(st.booleans()):
+        cu = [0] + sorted(set(data.draw(st.lists(st.integers(1, S - 1), max_size=5)))) + [S]
+    sch = api.ring_schedule(S, P, layout, causal, cu)
+    for (r, t), (j, live, _) in ref.pair_classes(S, P, layout, causal, cu).items():
+        i = r * P + t
+        assert sch["src"][i] == j
+        assert sch["live_pairs"][i] == live
+        assert sch["launched"][i] == (1 if live else 0)

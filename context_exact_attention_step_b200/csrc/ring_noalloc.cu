@@ -14,6 +14,9 @@
 // In host code `g_ring_scratch` only names the object; its device address is
 // looked up with cudaGetSymbolAddress once per device (on the first call made
 // with that device current) and that address is what the kernels receive.
+// The cached address belongs to the device's primary context: after a
+// cudaDeviceReset in the same process it would be stale, so the entry point
+// is not meant to be used across a reset.
 #include <cuda_runtime.h>
 
 #include <cstdio>

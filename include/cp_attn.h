@@ -186,7 +186,12 @@ cp_status cp_ulysses_permute(const void* in, void* out, int P, int S, int h, int
 
 /*
  * cp_zigzag_reorder -- natural token order <-> rank-major zigzag order
- * (rank i holds chunks i and 2P-1-i of 2P chunks of S/(2P) rows).  in/out are
+ * (rank i holds chunks i and 2P-1-i of 2P chunks of S/(2P) rows), the load
+ * balancing of causal Ring Attention: pairing an early chunk with a late one
+ * gives every rank the same share of the causal mask ("长上下文序列并行训练
+ * 深度解析" (mooersco) timeline, Striped / zigzag 负载均衡重排; the pages name
+ * the scheme without fixing the chunk pairing, which is taken as i with
+ * 2P-1-i, in that order inside the shard).  in/out are
  * [batch][S][row_bytes] byte arrays: use batch = 1, row_bytes = h*dh*elem for
  * Q/K/V/O, and batch = h, row_bytes = 4 for an fp32 LSE [h][S].
  * inverse = 0: natural -> zigzag; 1: zigzag -> natural.  Bit-exact.
@@ -210,7 +215,11 @@ cp_status cp_head_block_split(const void* in, void* out, int n, int h, int dh, i
 /*
  * cp_striped_reorder -- natural token order <-> rank-major striped order
  * (token t on rank t mod P, rank r's rows in position order: row r*S/P + a
- * holds position a*P + r).  in/out are [batch][S][row_bytes] byte arrays as
+ * holds position a*P + r), the Striped Attention balancing of causal Ring
+ * Attention: every rank holds positions spread evenly over the sequence, so
+ * every block pair is a (possibly one-key-shifted) local causal block
+ * ("长上下文序列并行训练深度解析" (mooersco) timeline, Striped / zigzag
+ * 负载均衡重排).  in/out are [batch][S][row_bytes] byte arrays as
  * for cp_zigzag_reorder.  inverse = 0: natural -> striped; 1: back.  Bit-exact.
  * Supported: S % P == 0; in and out must not overlap.
  */
@@ -436,7 +445,9 @@ cp_status cp_device_error(uint32_t* bits, int clear);
  *    rejected with CP_ERR_WORKSPACE and a message giving both sizes.
  *  - The first call on each device looks up the scratch address of that
  *    device (cudaGetSymbolAddress); make that first call before any stream
- *    capture begins.
+ *    capture begins.  The address is kept for the life of the process, so
+ *    the entry point must not be used after cudaDeviceReset (or any other
+ *    teardown of the device's primary context) in the same process.
  *  - All calls share the one scratch array per device and it keeps whatever
  *    the last call left there.  Calls whose GPU work overlaps in time (on
  *    different streams, or from different threads) race on it: order them on

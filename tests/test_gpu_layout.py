@@ -52,6 +52,38 @@ def test_ulysses_permute_full_size_q():
         assert torch.equal(back.view(torch.int16), x.view(torch.int16))
 
 
+def test_ulysses_permute_full_size_bit_exact():
+    """The whole 128K-token GQA workload (32 query / 8 KV heads, dh 128, P = 8):
+    seq->head of Q, K and V and head->seq of an fp32 O, every element against
+    the oracle's index formula."""
+    P, S, dh = 8, 131072, 128
+    n = S // P
+    for h, seed in ((32, 1), (8, 2), (8, 3)):
+        x = synth.normal((S, h, dh), seed, 0.5, torch.bfloat16).cuda()
+        y = api.ulysses_permute(x, P, "seq_to_head")
+        assert np.array_equal(bits(y), ref.ulysses_seq_to_head(bits(x).reshape(P, n, h, dh), P)), (h, seed)
+        del x, y
+    o = synth.normal((P, S, 32 // P, dh), 4, 1.0, torch.float32).cuda()
+    back = api.ulysses_permute(o, P, "head_to_seq")
+    assert np.array_equal(bits(back).reshape(P, n, 32, dh), ref.ulysses_head_to_seq(bits(o), P))
+
+
+def test_zigzag_full_size_bit_exact():
+    """The 64K-token zigzag workload (32 heads, dh 128, P = 8): the forward
+    reorder of a bf16 Q and the inverse of an fp32 O and LSE, every element
+    against the oracle's chunk order."""
+    P, S, h, dh = 8, 65536, 32, 128
+    q = synth.normal((S, h, dh), 1, 0.5, torch.bfloat16).cuda()
+    assert np.array_equal(bits(api.zigzag_reorder(q, P)), ref.zigzag_reorder(bits(q), P))
+    del q
+    o = synth.normal((S, h, dh), 5, 1.0, torch.float32).cuda()
+    assert np.array_equal(bits(api.zigzag_reorder(o, P, inverse=True)), ref.zigzag_restore(bits(o), P))
+    del o
+    lse = synth.normal((h, S), 6, 1.0, torch.float32).cuda()
+    got = api.zigzag_reorder(lse, P, inverse=True, seq_dim=1)
+    assert np.array_equal(bits(got), ref.zigzag_restore(bits(lse), P, axis=1))
+
+
 @pytest.mark.parametrize("P,S,shape,dtype", [
     (4, 64, (8, 128), torch.bfloat16),
     (8, 4096, (32, 128), torch.bfloat16),

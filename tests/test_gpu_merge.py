@@ -11,7 +11,8 @@ from _util import compare, f64
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("n,rows,h,dh", [(1, 37, 3, 128), (4, 300, 8, 128), (7, 129, 4, 64), (10, 1024, 32, 128)])
+@pytest.mark.parametrize("n,rows,h,dh", [(1, 37, 3, 128), (4, 300, 8, 128), (7, 129, 4, 64), (10, 1024, 32, 128),
+                                         (18, 100, 13, 64)])  # more partials than the kernel stages in shared memory
 def test_merge_matches_oracle(n, rows, h, dh):
     g = torch.Generator().manual_seed(n * 1000 + rows)
     o = [torch.randn(rows, h, dh, generator=g) for _ in range(n)]

@@ -487,6 +487,38 @@ def test_pair_classes_contiguous_and_zigzag():
         assert live == (2 * c * c + c if j == r else 2 * c * c)
 
 
+def test_ring_source_hand_table_p3():
+    """The rotation of "序列並行" concept page (compassingai), "Ring Attention 的
+    不同思路" steps 1-4: every rank starts with its own K/V block and at each
+    step passes the block it holds to the next rank and takes the previous
+    rank's.  For three ranks, written out by hand (rows: step t, columns: rank
+    r, entry: the shard rank r holds)."""
+    table = [[0, 1, 2],
+             [2, 0, 1],
+             [1, 2, 0]]
+    for t in range(3):
+        for r in range(3):
+            assert ref.ring_source(r, t, 3) == table[t][r], (r, t)
+
+
+def test_ring_source_matches_simulated_message_passing():
+    """Pass the blocks around explicitly (rank r sends what it holds to rank
+    r + 1 each step) and check that the oracle's schedule names the block each
+    rank holds, and that over P steps every rank meets every shard once."""
+    for P in range(1, 10):
+        held = list(range(P))            # step 0: every rank holds its own shard
+        seen = [set() for _ in range(P)]
+        for t in range(P):
+            for r in range(P):
+                assert ref.ring_source(r, t, P) == held[r], (P, r, t)
+                seen[r].add(held[r])
+            nxt = [None] * P
+            for r in range(P):
+                nxt[(r + 1) % P] = held[r]   # send to the next rank
+            held = nxt
+        assert all(sv == set(range(P)) for sv in seen)
+
+
 # ------------------------------------------------- planted mistakes are caught
 def test_pins_catch_planted_mistakes(monkeypatch):
     """Plant plausible mistakes in the oracle (on the CPU) and check that the

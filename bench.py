@@ -1,27 +1,39 @@
 #!/usr/bin/env python
 """Benchmark of the context-parallel exact attention hot path on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--pass fwd|bwd]
+                    [--impl ours|reference]
 
 One step = one pass of the hot path over one batch of synthetic input that is
-already resident in HBM.  For the default workload (ring attention forward,
-S=32768, 32 heads, dh=128, P=4 contiguous causal shards, bf16) a step is the
-ring-step schedule, the block-attention launch over all live block pairs and
-the fp32 LSE merge, all through ``cp_ring_attn_fwd``; zigzag workloads add the
-zigzag (or striped) reorder of Q, K, V and the inverse reorder of O and LSE;
-the Ulysses workload is seq->head transpose, per-group attention, head->seq
-transpose; the hybrid workload (usp_gqa_128k) is the zigzag reorder over the
-ring groups, the seq->head transpose over the Ulysses ranks, the ring block
-pairs of every head block, a merge that writes the head blocks back, and the
-inverse reorder.
+already resident in HBM.  With no --workload the line is headed by the
+packed-document ring forward: 131072 tokens of documents with lengths uniform
+in [1024, 32768] (seed 4), 32 heads, dh 128, P = 8 virtual ranks in the
+zigzag layout, bf16.  Its step is the zigzag reorder of Q, K, V, the ring-step
+schedule, the block-attention launch over all live block pairs, the fp32 LSE
+merge and the inverse reorder of O and LSE.  The same line carries, under one
+clock record, a sub-object per other workload:
+
+  ring_contig_32k    S=32768, P=4 contiguous causal (attention + merge)
+  ring_zigzag_64k    S=65536, P=8 zigzag causal (+ zigzag reorders)
+  ulysses_gqa_128k   S=131072, 32/8 heads, P=8 Ulysses (seq->head permutes,
+                     per-group attention, head->seq permute)
+  ring_striped_64k   S=65536, P=8 striped causal (+ striped reorders)
+  usp_gqa_128k       S=131072, 32/4 heads, Ulysses over 4 x ring over 2
+and the ring backward (dQ, dK, dV) of the 32K and packed-document workloads.
 
 The metric is causal-effective TFLOP/s (4 * dh * hq per admitted (q, k) pair,
-divided by the step time); the JSON line also carries the a2a-permute GB/s of
-the Ulysses transpose, the roofline of the dominant kernel, an end-to-end
-figure with host buffers, the CPU oracle baseline and the SM clocks.
+divided by the step time).  Each sub-object gives the attention kernel's own
+TFLOP/s and fraction of the measured bf16 peak, and the merge, reorder and
+permute kernels' GB/s and fraction of the measured HBM bandwidth, all timed
+with CUDA events on the launching stream.
 
-Under torchrun every rank runs its own independent problem (weak scaling; no
-data crosses GPUs), and the time is the max over ranks.
+--gpus N > 1 launches N ranks (one process per GPU, torchrun) unless the
+process already runs under torchrun; every rank times its own independent
+problem (weak scaling: the virtual ranks of the path never exchange data) and
+the time is the max over ranks.  With N > 1 the line also carries a `dist`
+object: the ring (64K tokens, zigzag) and Ulysses (128K tokens, 32/8 heads)
+run with the ranks on real GPUs, K/V rotating by NCCL send/recv and the
+Ulysses all-to-alls over NCCL, timed as the max over ranks.
 """
 from __future__ import annotations
 
@@ -30,6 +42,7 @@ import datetime
 import hashlib
 import json
 import os
+import socket
 import statistics
 import subprocess
 import sys
@@ -45,19 +58,25 @@ sys.path.insert(0, ROOT)
 METRIC = "ring-attn fwd TFLOP/s & % BF16 tensor peak; a2a-permute GB/s % HBM"
 METRIC_BWD = "ring-attn bwd TFLOP/s (causal-effective, 2.5x the forward's FLOP) & % BF16 tensor peak"
 
+HEADLINE = "varlen_zigzag_128k"
+SUITE = ["ring_contig_32k", "ring_zigzag_64k", "ulysses_gqa_128k", "ring_striped_64k", "usp_gqa_128k"]
+BWD_SUITE = ["ring_contig_32k", "varlen_zigzag_128k"]
+
 # DRAM traffic per launch of the block-attention kernel from an ncu capture,
-# keyed by the hash of the kernel source it was taken on (null once the
-# kernel changes).  Filled from profiles/ summaries.
+# keyed by (hash of the kernel source it was taken on, workload): a kernel
+# change makes the entry stale and the line reports null until the capture is
+# repeated.  Filled from the profiles/ summaries.
 ATTN_TRAFFIC = {
-    # profiles/attn_fwd_kernel_ring_contig_32k.md: 2.01 GB read + 1.33 GB written
-    # per launch on the 32K-token contiguous workload (one-pass capture).
-    ("e26710632bba45c5", "ring_contig_32k", 32768): 3.34e9,
 }
 
 
 def src_hash(path):
     with open(path, "rb") as f:
         return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def attn_src_hash():
+    return src_hash(os.path.join(ROOT, "context_exact_attention_step_b200", "csrc", "attn_fwd.cu"))
 
 
 # ----------------------------------------------------------------- helpers
@@ -72,16 +91,20 @@ def peaks():
 
 
 class Clocks:
-    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+    """Samples SM clocks and throttle reasons with nvidia-smi while the timed
+    regions run; start/stop may be called around several regions and the
+    summary covers every sample taken."""
 
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
     def __init__(self, index):
         self.index = index
         self.proc = None
         self.path = None
+        self.sm, self.mx, self.reasons = [], None, set()
 
     def start(self):
         fd, self.path = tempfile.mkstemp(suffix=".csv")
@@ -96,44 +119,49 @@ class Clocks:
 
     def stop(self):
         if self.proc is None:
-            return None
+            return
         time.sleep(0.1)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        self.proc = None
         with open(self.path) as f:
             for line in f:
                 parts = [x.strip() for x in line.split(",")]
                 if len(parts) < 9:
                     continue
                 try:
-                    sm.append(float(parts[1]))
-                    mx = float(parts[2])
+                    self.sm.append(float(parts[1]))
+                    self.mx = float(parts[2])
                 except ValueError:
                     continue
-                for n, val in zip(names, parts[5:9]):
+                for n, val in zip(self.NAMES, parts[5:9]):
                     if val.lower().startswith("active"):
-                        reasons.add(n)
+                        self.reasons.add(n)
         os.unlink(self.path)
-        if not sm:
+
+    def summary(self):
+        if not self.sm:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+        return {"sm_mhz": statistics.median(self.sm), "sm_max_mhz": self.mx, "reasons": sorted(self.reasons),
+                "samples": len(self.sm)}
 
 
-def dist_init():
+def dist_init(backend="nccl"):
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if ws > 1:
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    else:
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=60))
+    elif backend == "nccl":
         torch.cuda.set_device(0)
     return ws, rank, local
 
@@ -154,8 +182,41 @@ def max_over_ranks(x, ws):
     return float(t.item())
 
 
+def free_port():
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def relaunch(n):
+    """Runs this same command as n ranks under torchrun (one process per
+    GPU) and returns its exit status."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", "--master-port", str(free_port()), os.path.abspath(__file__),
+           *sys.argv[1:]]
+    return subprocess.run(cmd).returncode
+
+
+def ev():
+    e = torch.cuda.Event(enable_timing=True)
+    e.record()  # creates the CUDA handle
+    return e
+
+
+def tflops(flops, ms):
+    return flops / (ms * 1e-3) / 1e12
+
+
+def gbs(nbytes, ms):
+    return nbytes / (ms * 1e-3) / 1e9
+
+
 # ----------------------------------------------------------------- workloads
-def make_workload(name, seq_len=None, pass_="fwd"):
+def make_workload(name, seq_len=None, pass_="fwd", host=False):
+    """Inputs of a workload on the device and its step.  The step takes an
+    optional list of four events recorded around the layout kernels that run
+    outside the library's composite call (before: the forward reorder of Q,
+    K, V; after: the inverse reorder of O and LSE)."""
     from context_exact_attention_step_b200 import api, synth
     cfg = dict(synth.CONFIGS[name])
     if seq_len:
@@ -171,17 +232,23 @@ def make_workload(name, seq_len=None, pass_="fwd"):
     w = dict(name=name, cfg=cfg, S=S, hq=hq, hkv=hkv, dh=dh, P=P, layout=layout, cu=cu, dtype=dtype)
     w["pairs"] = api.count_live_pairs(S, True, cu)
     w["flops"] = 4.0 * dh * hq * w["pairs"]
-    w["host"] = [t.pin_memory() for t in (q, k, v)]
+    if host:
+        w["host"] = [t.pin_memory() for t in (q, k, v)]
     qd, kd, vd = (t.to(dev) for t in (q, k, v))
+    del q, k, v
     w["in"] = (qd, kd, vd)
     o = torch.empty((S, hq, dh), device=dev, dtype=torch.float32)
     lse = torch.empty((hq, S), device=dev, dtype=torch.float32)
     w["out"] = (o, lse)
+    w["reorder_bytes"] = 0
+    mark = lambda marks, i: marks[i].record() if marks else None
     if layout == "ulysses":
         ws = torch.empty(api.ulysses_attn_workspace_size(S, hq, hkv, dh, P), device=dev, dtype=torch.uint8)
 
-        def step():
+        def step(marks=None):
             api.ulysses_attn_fwd(qd, kd, vd, P, True, o=o, lse=lse, workspace=ws)
+        # seq->head of Q, K, V (bf16) and head->seq of O (fp32): read + write once
+        w["permute_bytes"] = 2 * (sum(t.numel() * t.element_size() for t in (qd, kd, vd)) + o.numel() * 4)
     elif layout == "usp":
         Pr, Pu, rl = cfg["Pr"], cfg["Pu"], cfg["ring_layout"]
         ws = torch.empty(api.usp_attn_workspace_size(S, hq, hkv, dh, Pr, Pu, rl, True), device=dev,
@@ -191,15 +258,21 @@ def make_workload(name, seq_len=None, pass_="fwd"):
         lz = torch.empty_like(lse)
         reorder = api.zigzag_reorder if rl == "zigzag" else api.striped_reorder
 
-        def step():
+        def step(marks=None):
+            mark(marks, 0)
             reorder(qd, Pr, out=qz)
             reorder(kd, Pr, out=kz)
             reorder(vd, Pr, out=vz)
+            mark(marks, 1)
             api.usp_attn_fwd(qz, kz, vz, Pr, Pu, rl, True, o=oz, lse=lz, workspace=ws)
+            mark(marks, 2)
             reorder(oz, Pr, inverse=True, out=o)
             reorder(lz, Pr, inverse=True, seq_dim=1, out=lse)
+            mark(marks, 3)
+        w["reorder_bytes"] = 2 * sum(t.numel() * t.element_size() for t in (qd, kd, vd, o, lse))
     else:
         cu_dev = torch.tensor(cu, dtype=torch.int32, device=dev) if cu is not None else None
+        w["cu_dev"] = cu_dev
         ws = torch.empty(max(256, api.ring_attn_workspace_size(S, hq, hkv, dh, P, layout, True, dtype, cu)),
                          device=dev, dtype=torch.uint8)
         if layout in ("zigzag", "striped"):
@@ -208,18 +281,24 @@ def make_workload(name, seq_len=None, pass_="fwd"):
             lz = torch.empty_like(lse)
             reorder = api.zigzag_reorder if layout == "zigzag" else api.striped_reorder
 
-            def step():
+            def step(marks=None):
+                mark(marks, 0)
                 reorder(qd, P, out=qz)
                 reorder(kd, P, out=kz)
                 reorder(vd, P, out=vz)
+                mark(marks, 1)
                 api.ring_attn_fwd(qz, kz, vz, P, layout, True, cu, cu_dev, o=oz, lse=lz, workspace=ws)
+                mark(marks, 2)
                 reorder(oz, P, inverse=True, out=o)
                 reorder(lz, P, inverse=True, seq_dim=1, out=lse)
+                mark(marks, 3)
+            w["reorder_bytes"] = 2 * sum(t.numel() * t.element_size() for t in (qd, kd, vd, o, lse))
         else:
-            def step():
+            def step(marks=None):
                 api.ring_attn_fwd(qd, kd, vd, P, layout, True, cu, cu_dev, o=o, lse=lse, workspace=ws)
+    w["fwd_ws"] = ws
     if pass_ == "bwd":
-        make_bwd_step(w, api, synth, dev, ws)
+        make_bwd_step(w, api, synth, dev, ws, host)
     else:
         w["step"] = step
         w["ws_bytes"] = ws.numel()
@@ -227,7 +306,7 @@ def make_workload(name, seq_len=None, pass_="fwd"):
     return w
 
 
-def make_bwd_step(w, api, synth, dev, fwd_ws):
+def make_bwd_step(w, api, synth, dev, fwd_ws, host):
     """Backward step of a ring workload: cp_ring_attn_bwd on inputs already in
     the rank-major shard order, with O and LSE from one forward call made here
     (outside any timed region) and a seeded upstream gradient dO."""
@@ -238,15 +317,13 @@ def make_bwd_step(w, api, synth, dev, fwd_ws):
     S, hq, hkv, dh = w["S"], w["hq"], w["hkv"], w["dh"]
     if w["dtype"] != torch.bfloat16:
         raise SystemExit("--pass bwd takes bf16 workloads")
-    do = synth.normal((S, hq, dh), synth.SEED_DO, 0.5)
+    do = synth.normal((S, hq, dh), synth.SEED_DO, 0.5).to(dev)
     if layout != "contiguous":
         reorder = api.zigzag_reorder if layout == "zigzag" else api.striped_reorder
-        qd, kd, vd = (reorder(t, P) for t in (qd, kd, vd))
-        do = reorder(do.to(dev), P).cpu()
-    cu_dev = torch.tensor(cu, dtype=torch.int32, device=dev) if cu is not None else None
+        qd, kd, vd, do = (reorder(t, P) for t in (qd, kd, vd, do))
+    cu_dev = w.get("cu_dev")
     o, lse = w["out"]
     api.ring_attn_fwd(qd, kd, vd, P, layout, True, cu, cu_dev, o=o, lse=lse, workspace=fwd_ws)
-    dod = do.to(dev)
     dq = torch.empty((S, hq, dh), device=dev, dtype=torch.float32)
     dk = torch.empty((S, hkv, dh), device=dev, dtype=torch.float32)
     dv = torch.empty_like(dk)
@@ -254,13 +331,14 @@ def make_bwd_step(w, api, synth, dev, fwd_ws):
                      dtype=torch.uint8)
     torch.cuda.synchronize()
 
-    def step():
-        api.ring_attn_bwd(qd, kd, vd, o, lse, dod, P, layout, True, cu, cu_dev, dq=dq, dk=dk, dv=dv, workspace=ws)
+    def step(marks=None):
+        api.ring_attn_bwd(qd, kd, vd, o, lse, do, P, layout, True, cu, cu_dev, dq=dq, dk=dk, dv=dv, workspace=ws)
 
     w["step"] = step
     w["ws_bytes"] = ws.numel()
-    w["host"] = [t.cpu().pin_memory() for t in (qd, kd, vd, o, lse, dod)]
-    w["in"] = (qd, kd, vd, o, lse, dod)
+    if host:
+        w["host"] = [t.cpu().pin_memory() for t in (qd, kd, vd, o, lse, do)]
+    w["in"] = (qd, kd, vd, o, lse, do)
     w["out"] = (dq, dk, dv)
     w["fwd_flops"] = w["flops"]
     # five score-sized products (S, dP, dV, dK, dQ) against the forward's two
@@ -268,15 +346,17 @@ def make_bwd_step(w, api, synth, dev, fwd_ws):
 
 
 def time_steps(w, steps, warmup, ws):
+    """W untimed steps, then exactly K steps bracketed by a barrier and a
+    synchronize on both sides.  Inside the timed region every step also
+    records the library's phase events (attention begin / end, merge end; for
+    the backward the dQ / dK-dV boundary) and the layout-kernel marks."""
     from context_exact_attention_step_b200 import api
     step = w["step"]
     for _ in range(warmup):
         step()
     torch.cuda.synchronize()
-    ev = lambda: torch.cuda.Event(enable_timing=True)
-    ab, ae, me = [ev() for _ in range(steps)], [ev() for _ in range(steps)], [ev() for _ in range(steps)]
-    for e in ab + ae + me:
-        e.record()  # creates the CUDA handles
+    n_ev = 9
+    evs = [[ev() for _ in range(n_ev)] for _ in range(steps)]
     torch.cuda.synchronize()
     barrier(ws)
     torch.cuda.synchronize()
@@ -284,24 +364,82 @@ def time_steps(w, steps, warmup, ws):
     n0 = api.kernel_launch_count()
     t0.record()
     for i in range(steps):
-        api.set_profile_events(ab[i], ae[i], me[i])
-        step()
+        e = evs[i]
+        e[0].record()
+        api.set_profile_events(e[1], e[2], e[3])
+        step(e[4:8])
+        e[8].record()
     t1.record()
     api.set_profile_events(None, None, None)
     torch.cuda.synchronize()
     launches = api.kernel_launch_count() - n0
     barrier(ws)
-    total_ms = t0.elapsed_time(t1)
-    attn_ms = [a.elapsed_time(b) for a, b in zip(ab, ae)]
-    if w.get("pass") == "bwd":  # merge_end marks the boundary between the dQ and dK/dV kernels
-        merge_ms = {"dq": [a.elapsed_time(b) for a, b in zip(ab, me)],
-                    "dkdv": [a.elapsed_time(b) for a, b in zip(me, ae)]}
-    else:
-        merge_ms = [a.elapsed_time(b) for a, b in zip(ae, me)] if w["layout"] != "ulysses" else []
     err = api.device_error()
     if err:
         raise RuntimeError(f"device error word {err:#x}: a kernel gave up waiting")
-    return total_ms, attn_ms, merge_ms, launches
+    has_marks = w["reorder_bytes"] > 0 and w.get("pass") != "bwd"
+    r = {"ms": t0.elapsed_time(t1) / steps, "launches": launches}
+    # per step: e0 start, e1 attention begin, e2 attention end, e3 merge end
+    # (bwd: dQ end), e4..e7 reorder marks, e8 end
+    r["attn"] = [e[1].elapsed_time(e[2]) for e in evs]
+    if w.get("pass") == "bwd":
+        r["dq"] = [e[1].elapsed_time(e[3]) for e in evs]
+        r["dkdv"] = [e[3].elapsed_time(e[2]) for e in evs]
+    elif w["layout"] == "ulysses":  # permutes: before and after the attention, inside the call
+        r["permute"] = [e[0].elapsed_time(e[1]) + e[2].elapsed_time(e[8]) for e in evs]
+    else:
+        r["merge"] = [e[2].elapsed_time(e[3]) for e in evs]
+    if has_marks:
+        r["reorder"] = [e[4].elapsed_time(e[5]) + e[6].elapsed_time(e[7]) for e in evs]
+    return r
+
+
+def merge_bytes(w):
+    """Algorithmic bytes of the merge: every live partial (O fp32 + LSE) read
+    once, the output O and LSE written once."""
+    from context_exact_attention_step_b200 import api
+    cfg = w["cfg"]
+    if w["layout"] == "usp":  # Pu rings of Pr ranks over hq/Pu heads each
+        sch = api.ring_schedule(w["S"], cfg["Pr"], cfg["ring_layout"], True, w["cu"])
+    else:
+        sch = api.ring_schedule(w["S"], w["P"], w["layout"], True, w["cu"])
+    rows = int(sch["q_rows"].sum())
+    per_row = w["hq"] * (w["dh"] + 1) * 4
+    return rows * per_row + w["S"] * per_row
+
+
+def summarize(w, r, pk, ws):
+    """Per-workload figures: step, attention kernel, merge / reorder / permute
+    kernels; times are means over the timed steps, max over ranks."""
+    ms = max_over_ranks(r["ms"], ws)
+    out = {"ms_per_step": ms, "tflops": tflops(w["flops"] * ws, ms), "flops_per_step": w["flops"],
+           "admitted_pairs": w["pairs"]}
+    am = max_over_ranks(statistics.mean(r["attn"]), ws)
+    if w.get("pass") == "bwd":
+        out["kernels"] = {"ms": am, "tflops": tflops(w["flops"], am), "frac": tflops(w["flops"], am) / pk["bf16"]}
+        for name, gemms in (("dq", 3), ("dkdv", 4)):
+            kms = max_over_ranks(statistics.mean(r[name]), ws)
+            ex = gemms / 2.0 * w["fwd_flops"]  # tensor work the kernel executes (S, dP, dQ / S^T, dP^T, dV, dK)
+            out[name] = {"ms": kms, "executed_tflops": tflops(ex, kms), "executed_frac": tflops(ex, kms) / pk["bf16"]}
+        return out
+    out["attn"] = {"ms": am, "tflops": tflops(w["flops"], am), "frac": tflops(w["flops"], am) / pk["bf16"],
+                   "frac_of_sustained": tflops(w["flops"], am) / pk["bf16_sus"],
+                   "traffic": ATTN_TRAFFIC.get((attn_src_hash(), w["name"]))}
+    if "merge" in r:
+        mb = merge_bytes(w)
+        mm = max_over_ranks(statistics.mean(r["merge"]), ws)
+        out["merge"] = {"ms": mm, "gbs": gbs(mb, mm), "frac_hbm": gbs(mb, mm) / pk["hbm_gbs"], "bytes": mb}
+    if "reorder" in r:
+        rm = max_over_ranks(statistics.mean(r["reorder"]), ws)
+        rb = w["reorder_bytes"]
+        out["reorder"] = {"ms": rm, "gbs": gbs(rb, rm), "frac_hbm": gbs(rb, rm) / pk["hbm_gbs"], "bytes": rb,
+                          "what": f"{w['cfg'].get('ring_layout', w['layout'])} reorder of Q, K, V and inverse of O, LSE"}
+    if "permute" in r:
+        pm = max_over_ranks(statistics.mean(r["permute"]), ws)
+        pb = w["permute_bytes"]
+        out["permute"] = {"ms": pm, "gbs": gbs(pb, pm), "frac_hbm": gbs(pb, pm) / pk["hbm_gbs"], "bytes": pb,
+                          "what": "seq->head of Q, K, V (bf16) + head->seq of O (fp32)"}
+    return out
 
 
 def time_e2e(w, steps):
@@ -320,9 +458,9 @@ def time_e2e(w, steps):
     stage_in = [[torch.empty_like(t) for t in devs_in] for _ in range(2)]
     stage_out = [[torch.empty_like(t) for t in devs_out] for _ in range(2)]
     s_h, s_c, s_d = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
-    ev = lambda: torch.cuda.Event()
-    in_ready, in_free = [ev(), ev()], [ev(), ev()]
-    out_ready, out_free = [ev(), ev()], [ev(), ev()]
+    plain = lambda: torch.cuda.Event()
+    in_ready, in_free = [plain(), plain()], [plain(), plain()]
+    out_ready, out_free = [plain(), plain()], [plain(), plain()]
 
     def one(i):
         slot = i % 2
@@ -365,42 +503,6 @@ def time_e2e(w, steps):
     h2d = sum(t.numel() * t.element_size() for t in hosts_in)
     d2h = sum(t.numel() * t.element_size() for t in hosts_out[0])
     return ms, h2d, d2h
-
-
-def time_permute(reps=20):
-    """a2a-permute GB/s of the Ulysses transposes on the 128K-token GQA
-    workload: seq->head of Q (32 heads), K and V (8 heads), head->seq of the
-    fp32 O; bytes = read + write of every element once."""
-    from context_exact_attention_step_b200 import api, synth
-    S, hq, hkv, dh, P = 131072, 32, 8, 128, 8
-    dev = torch.device("cuda")
-    q = synth.normal((S, hq, dh), 1, 0.5).to(dev)
-    k = synth.normal((S, hkv, dh), 2, 0.5).to(dev)
-    v = synth.normal((S, hkv, dh), 3, 0.5).to(dev)
-    oh = torch.randn((P, S, hq // P, dh), device=dev, dtype=torch.float32)
-    qh = torch.empty((P, S, hq // P, dh), device=dev, dtype=torch.bfloat16)
-    kh = torch.empty((P, S, hkv // P, dh), device=dev, dtype=torch.bfloat16)
-    vh = torch.empty_like(kh)
-    o = torch.empty((S, hq, dh), device=dev, dtype=torch.float32)
-
-    def run():
-        api.ulysses_permute(q, P, "seq_to_head", out=qh)
-        api.ulysses_permute(k, P, "seq_to_head", out=kh)
-        api.ulysses_permute(v, P, "seq_to_head", out=vh)
-        api.ulysses_permute(oh, P, "head_to_seq", out=o)
-
-    for _ in range(3):
-        run()
-    torch.cuda.synchronize()
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t0.record()
-    for _ in range(reps):
-        run()
-    t1.record()
-    torch.cuda.synchronize()
-    ms = t0.elapsed_time(t1) / reps
-    nbytes = 2 * sum(t.numel() * t.element_size() for t in (q, k, v, oh))
-    return dict(gbs=nbytes / (ms * 1e-3) / 1e9, ms=ms, bytes=nbytes)
 
 
 # ----------------------------------------------------------------- multi-GPU ring, rank by rank
@@ -502,6 +604,62 @@ def time_per_rank(w, reps=5):
     }
 
 
+# ----------------------------------------------------------------- real multi-GPU legs
+def time_dist(ws, rank, steps, warmup):
+    """The ring and Ulysses with the ranks on real GPUs (``distributed``):
+    every rank holds shard `rank` of the sequence; K/V rotate by NCCL
+    send/recv into local buffers (ring) or move by NCCL all-to-all (Ulysses);
+    no kernel reads another GPU's memory.  Time = max over ranks of the
+    CUDA-event time of K calls."""
+    from context_exact_attention_step_b200 import api, synth
+    from context_exact_attention_step_b200 import distributed as D
+    import torch.distributed as dist
+    dev = torch.device("cuda")
+    out = {}
+    legs = [("ring_zigzag_64k", "ring"), ("ulysses_gqa_128k", "ulysses")]
+    for name, kind in legs:
+        cfg = synth.CONFIGS[name]
+        S, hq, hkv, dh = cfg["S"], cfg["hq"], cfg["hkv"], cfg["dh"]
+        if kind == "ring" and S % (2 * ws):
+            continue
+        if kind == "ulysses" and hkv % ws:
+            out[kind] = {"skipped": f"{ws} ranks do not divide the {hkv} KV heads"}
+            continue
+        q, k, v = (t.to(dev) for t in synth.qkv(S, hq, hkv, dh, std=cfg["std"], dtype=torch.bfloat16))
+        n = S // ws
+        if kind == "ring":
+            q, k, v = (api.zigzag_reorder(t, ws) for t in (q, k, v))
+        qs, ks, vs = (t[rank * n:(rank + 1) * n].contiguous() for t in (q, k, v))
+        del q, k, v
+        torch.cuda.empty_cache()
+        if kind == "ring":
+            call = lambda: D.ring_attn_fwd_dist(qs, ks, vs, "zigzag", True)
+        else:
+            call = lambda: D.ulysses_attn_fwd_dist(qs, ks, vs, True)
+        for _ in range(warmup):
+            call()
+        torch.cuda.synchronize()
+        barrier(ws)
+        torch.cuda.synchronize()
+        a, b = ev(), ev()
+        a.record()
+        for _ in range(steps):
+            call()
+        b.record()
+        torch.cuda.synchronize()
+        barrier(ws)
+        ms = max_over_ranks(a.elapsed_time(b) / steps, ws)
+        flops = 4.0 * dh * hq * S * (S + 1) / 2
+        out[kind] = {"workload": name, "ranks": ws, "S": S, "ms_per_step": ms, "tflops": tflops(flops, ms),
+                     "tflops_per_gpu": tflops(flops, ms) / ws,
+                     "exchange": ("K/V of the shard to rank r+1 per ring step (NCCL send/recv, posted before the "
+                                  "step's block attention)" if kind == "ring" else
+                                  "all-to-all of Q, K, V to head blocks and of O, LSE back (NCCL)")}
+        del qs, ks, vs
+        torch.cuda.empty_cache()
+    return out
+
+
 # ----------------------------------------------------------------- CPU oracle
 def oracle_sample_rate(w, target_s=12.0, max_rows=1024, seed=0, bwd=False):
     """Times the fp64 oracle on a bounded sample of the same workload: batches
@@ -541,6 +699,15 @@ def oracle_sample_rate(w, target_s=12.0, max_rows=1024, seed=0, bwd=False):
 
 
 # ----------------------------------------------------------------- arms
+def workload_identity(name, cfg, pairs, bwd):
+    return {"workload": name, **{k_: cfg[k_] for k_ in ("S", "hq", "hkv", "dh", "P", "layout")},
+            "causal": True, "input_dtype": cfg["dtype"], "admitted_pairs": pairs,
+            "flops_per_step": (10.0 if bwd else 4.0) * cfg["dh"] * cfg["hq"] * pairs,
+            **({k_: cfg[k_] for k_ in ("Pr", "Pu", "ring_layout")} if cfg["layout"] == "usp" else {}),
+            **({"documents": "lengths uniform in [%d, %d], seed 4, last one truncated" % (cfg["doc_lo"], cfg["doc_hi"])}
+               if cfg.get("varlen") else {})}
+
+
 def run_reference(args, ws, rank):
     """Reference arm: the fp64 CPU oracle as it stands, on the same workload,
     metric and unit; every step is a bounded sample of 32 query rows."""
@@ -548,7 +715,7 @@ def run_reference(args, ws, rank):
         return
     from context_exact_attention_step_b200 import synth
     from oracle import ref
-    name = args.workload
+    name = args.workload or HEADLINE
     cfg = synth.CONFIGS[name]
     S, hq, hkv, dh = cfg["S"], cfg["hq"], cfg["hkv"], cfg["dh"]
     dtype = torch.float32 if cfg["dtype"] == "fp32" else torch.bfloat16
@@ -577,10 +744,7 @@ def run_reference(args, ws, rank):
     # closed form: S(S+1)/2, or the sum of L(L+1)/2 over the documents)
     lens = np.diff(np.asarray(cu, dtype=np.int64)) if cu is not None else np.array([S], dtype=np.int64)
     pairs = int((lens * (lens + 1) // 2).sum())
-    ref_config = {"workload": name, **{k_: cfg[k_] for k_ in ("S", "hq", "hkv", "dh", "P", "layout")},
-                  "causal": True, "input_dtype": cfg["dtype"], "admitted_pairs": pairs,
-                  "flops_per_step": (10.0 if bwd else 4.0) * dh * hq * pairs,
-                  **({k_: cfg[k_] for k_ in ("Pr", "Pu", "ring_layout")} if cfg["layout"] == "usp" else {})}
+    ref_config = workload_identity(name, cfg, pairs, bwd)
     if bwd:
         ref_config["pass"] = "backward: the gradient of the sampled query rows"
     for _ in range(args.warmup):
@@ -603,111 +767,158 @@ def run_reference(args, ws, rank):
     print(json.dumps(line), flush=True)
 
 
+def free(w):
+    for key in ("in", "out", "host", "fwd_ws", "step", "cu_dev"):
+        w.pop(key, None)
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+
 def run_ours(args, ws, rank, local):
-    from context_exact_attention_step_b200 import api
     from context_exact_attention_step_b200 import build as _build
     _build.build()
     pk = peaks()
-    w = make_workload(args.workload, args.seq_len, args.pass_)
     bwd = args.pass_ == "bwd"
+    name = args.workload or HEADLINE
+    suite = args.workload is None and not args.no_suite and not bwd
     clocks = Clocks(local)
+
+    w = make_workload(name, args.seq_len, args.pass_, host=True)
     clocks.start()
-    total_ms, attn_ms, merge_ms, launches = time_steps(w, args.steps, args.warmup, ws)
-    ck = clocks.stop()
-    ms_step = max_over_ranks(total_ms / args.steps, ws)
-    value = w["flops"] * ws / (ms_step * 1e-3) / 1e12
-    attn_avg = statistics.mean(attn_ms)
-    attn_tf = w["flops"] / (attn_avg * 1e-3) / 1e12
-    traffic = ATTN_TRAFFIC.get((src_hash(os.path.join(ROOT, "context_exact_attention_step_b200", "csrc",
-                                                      "attn_fwd.cu")), w["name"], w["S"]))
+    r = time_steps(w, args.steps, args.warmup, ws)
+    clocks.stop()
+    head = summarize(w, r, pk, ws)
     e2e_ms, h2d, d2h = time_e2e(w, args.e2e_steps)
     e2e_ms = max_over_ranks(e2e_ms, ws)
-    perm = time_permute() if not (args.no_permute or bwd) else None
-    cfg = w["cfg"]
+    per_rank = time_per_rank(w) if args.per_rank else None
+    ident = workload_identity(name, w["cfg"], w["pairs"], bwd)
+    ident["S"] = w["S"]
+    cpu = oracle_sample_rate(w, bwd=bwd) if (rank == 0 and ws == 1 and not args.no_cpu_baseline) else None
+    head_flops = w["flops"]
+    free(w)
+
+    configs, bwd_configs = {}, {}
+    if suite:
+        for sname in SUITE:
+            sw = make_workload(sname)
+            clocks.start()
+            sr = time_steps(sw, args.steps, args.warmup, ws)
+            clocks.stop()
+            configs[sname] = summarize(sw, sr, pk, ws)
+            free(sw)
+        for sname in BWD_SUITE:
+            sw = make_workload(sname, pass_="bwd")
+            clocks.start()
+            sr = time_steps(sw, args.steps, args.warmup, ws)
+            clocks.stop()
+            bwd_configs[sname] = summarize(sw, sr, pk, ws)
+            free(sw)
+    dist_legs = time_dist(ws, rank, args.steps, args.warmup) if ws > 1 and not args.no_dist else None
+
+    if bwd:
+        kern = head["kernels"]
+        roof = {"bound": "tensor", "kernel": "attn_bwd_dq_kernel + attn_bwd_dkdv_kernel", "achieved": kern["tflops"],
+                "peak": pk["bf16"], "unit": "TFLOP/s", "frac": kern["frac"], "traffic": None,
+                "peak_source": pk["source"] + " burst bf16", "ms": kern["ms"]}
+    else:
+        a = head["attn"]
+        roof = {"bound": "tensor", "kernel": "attn_fwd_kernel", "achieved": a["tflops"], "peak": pk["bf16"],
+                "unit": "TFLOP/s", "frac": a["frac"], "traffic": a["traffic"],
+                "peak_source": pk["source"] + " burst bf16", "frac_of_sustained": a["frac_of_sustained"],
+                "frac_of_nominal_2250": a["tflops"] / 2250.0, "attn_ms": a["ms"]}
     line = {
-        "metric": METRIC_BWD if bwd else METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w["name"], "S": w["S"], "hq": w["hq"], "hkv": w["hkv"], "dh": w["dh"], "P": w["P"],
-                   "layout": w["layout"], "causal": True, "input_dtype": cfg["dtype"],
-                   "admitted_pairs": w["pairs"], "flops_per_step": w["flops"],
-                   "l2": "inputs larger than L2 (Q+K+V %.0f MB, partials %.0f MB)" % (
-                       sum(t.numel() * t.element_size() for t in w["in"]) / 1e6, w["ws_bytes"] / 1e6),
-                   "per_gpu": "independent problem per GPU",
-                   **({k_: cfg[k_] for k_ in ("Pr", "Pu", "ring_layout")} if w["layout"] == "usp" else {})},
-        "roofline": {"bound": "tensor",
-                     "kernel": "attn_bwd_dq_kernel + attn_bwd_dkdv_kernel" if bwd else "attn_fwd_kernel",
-                     "achieved": attn_tf, "peak": pk["bf16"],
-                     "unit": "TFLOP/s", "frac": attn_tf / pk["bf16"], "traffic": None if bwd else traffic,
-                     "peak_source": pk["source"] + " burst bf16", "frac_of_sustained": attn_tf / pk["bf16_sus"],
-                     "frac_of_nominal_2250": attn_tf / 2250.0, "attn_ms": attn_avg},
-        "e2e": {"value": w["flops"] * ws / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+        "metric": METRIC_BWD if bwd else METRIC, "value": head["tflops"], "unit": "TFLOP/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {**ident,
+                   "l2": "inputs larger than L2 (%.0f MB read per step, no flush needed)" % (h2d / 1e6),
+                   "per_gpu": "independent problem per GPU (the P virtual ranks of one problem share a GPU)",
+                   **({"pass": "backward (prep + dQ kernel + dK/dV kernel), inputs in shard order"} if bwd else {})},
+        "roofline": roof,
+        "e2e": {"value": tflops(head_flops * ws, e2e_ms), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "pipelining": "H2D of step i+1 and D2H of step i-1 overlap step i (two staging slots)"},
-        "gpu_launches": int(launches),
-        "clocks": ck,
+        "gpu_launches": int(r["launches"]),
+        "clocks": clocks.summary(),
     }
-    if bwd:
-        # per kernel: time and the tensor work each one executes (dQ side: S,
-        # dP, dQ; dK/dV side: S^T, dP^T, dV, dK; two FLOP per multiply-add)
-        for name, gemms in (("dq", 3), ("dkdv", 4)):
-            kms = statistics.mean(merge_ms[name])
-            ex = gemms / 2.0 * w["fwd_flops"]
-            line["bwd_" + name] = {"ms": kms, "executed_tflops": ex / (kms * 1e-3) / 1e12,
-                                   "executed_frac": ex / (kms * 1e-3) / 1e12 / pk["bf16"]}
-        line["config"]["pass"] = "backward (prep + dQ kernel + dK/dV kernel), inputs in shard order"
-    elif merge_ms:
-        mb = merge_bytes(w)
-        mms = statistics.mean(merge_ms)
-        line["merge"] = {"ms": mms, "gbs": mb / (mms * 1e-3) / 1e9, "frac_hbm": mb / (mms * 1e-3) / 1e9 / pk["hbm_gbs"],
-                         "bytes": mb}
-    if perm:
-        line["a2a_permute"] = {"gbs": perm["gbs"], "frac_hbm": perm["gbs"] / pk["hbm_gbs"], "ms": perm["ms"],
-                               "bytes": perm["bytes"], "workload": "ulysses_gqa_128k Q,K,V seq->head + fp32 O head->seq"}
-    if args.per_rank:
-        line["per_rank"] = time_per_rank(w)
-    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = oracle_sample_rate(w, bwd=bwd)
+    for key in ("merge", "reorder", "permute", "dq", "dkdv"):
+        if key in head:
+            line[key] = head[key]
+    if configs:
+        line["configs"] = configs
+        if "ulysses_gqa_128k" in configs:
+            p = configs["ulysses_gqa_128k"]["permute"]
+            line["a2a_permute"] = {**p, "workload": "ulysses_gqa_128k"}
+    if bwd_configs:
+        line["bwd"] = bwd_configs
+    if dist_legs:
+        line["dist"] = dist_legs
+    if per_rank:
+        line["per_rank"] = per_rank
+    if cpu:
+        line["cpu_baseline"] = cpu
     if rank == 0:
         print(json.dumps(line), flush=True)
 
 
-def merge_bytes(w):
-    """Algorithmic bytes of the merge: every live partial (O fp32 + LSE) read
-    once, the output O and LSE written once."""
-    from context_exact_attention_step_b200 import api
-    cfg = w["cfg"]
-    if w["layout"] == "usp":  # Pu rings of Pr ranks over hq/Pu heads each
-        sch = api.ring_schedule(w["S"], cfg["Pr"], cfg["ring_layout"], True, w["cu"])
+def check_launch(ws, rank):
+    """--check-launch: the launcher and the rank bookkeeping without a GPU
+    (gloo): every rank reports, rank 0 prints one line."""
+    import torch.distributed as dist
+    if ws > 1:
+        t = torch.tensor([rank], dtype=torch.int64)
+        got = [torch.zeros(1, dtype=torch.int64) for _ in range(ws)]
+        dist.all_gather(got, t)
+        ranks = [int(x.item()) for x in got]
+        slowest = max_over_ranks(1.0 + rank, ws)
+        barrier(ws)
     else:
-        sch = api.ring_schedule(w["S"], w["P"], w["layout"], True, w["cu"])
-    rows = int(sch["q_rows"].sum())
-    per_row = w["hq"] * (w["dh"] + 1) * 4
-    return rows * per_row + w["S"] * per_row
+        ranks, slowest = [0], 1.0
+    if rank == 0:
+        print(json.dumps({"n_gpus": ws, "ranks": ranks, "max_over_ranks": slowest}), flush=True)
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--e2e-steps", type=int, default=8)
-    ap.add_argument("--workload", default="ring_contig_32k")
+    ap.add_argument("--e2e-steps", type=int, default=6)
+    ap.add_argument("--workload", default=None,
+                    help=f"time only this workload (default: {HEADLINE} plus the per-config suite)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--no-permute", action="store_true")
     ap.add_argument("--pass", dest="pass_", default="fwd", choices=["fwd", "bwd"],
                     help="bwd: time the ring backward (dQ, dK, dV) of a ring workload instead of the forward")
+    ap.add_argument("--no-suite", action="store_true", help="headline workload only")
+    ap.add_argument("--no-dist", action="store_true", help="skip the multi-GPU ring / Ulysses legs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--per-rank", action="store_true",
                     help="also time each rank's kernel work of the multi-GPU ring (ring workloads)")
     ap.add_argument("--seq-len", type=int, default=None,
                     help="override the workload's sequence length (smaller cases for profiler captures)")
+    ap.add_argument("--check-launch", action="store_true", help=argparse.SUPPRESS)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.gpus < 1:
+        ap.error("--gpus must be at least 1")
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        sys.exit(relaunch(args.gpus))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world != args.gpus:
+        sys.stderr.write(f"bench.py: --gpus {args.gpus} but the launcher started {world} ranks\n")
+        sys.exit(2)
+    if args.check_launch:
+        ws, rank, _ = dist_init("gloo")
+        try:
+            check_launch(ws, rank)
+        finally:
+            if ws > 1:
+                import torch.distributed as dist
+                dist.destroy_process_group()
+        return
     if args.impl == "reference":
-        rank = int(os.environ.get("RANK", "0"))
-        run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), rank)
+        run_reference(args, world, int(os.environ.get("RANK", "0")))
         return
     ws, rank, local = dist_init()
     try:

@@ -9,6 +9,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <climits>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -25,7 +26,8 @@ namespace cp {
 cudaError_t launch_attn(int dh, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                         const cp_attn_plan& plan, cudaStream_t stream);
 cudaError_t attn_err_word(uint32_t** dev_ptr);
-cudaError_t launch_merge(const cp_merge_plan& plan, int max_rows, cudaStream_t stream);
+cudaError_t launch_merge(const cp_merge_plan& plan, int total_ctas, cudaStream_t stream);
+int merge_task_ctas(int rows, int h);
 cudaError_t launch_ulysses(const void* in, void* out, int P, int n, size_t chunk_bytes, int dir, cudaStream_t st);
 cudaError_t launch_zigzag(const void* in, void* out, int P, int batch, size_t chunk_bytes, int inverse,
                           cudaStream_t st);
@@ -142,6 +144,7 @@ struct PairIn {
   float* lse;
   int lse_ld;
   bool reverse;
+  int block = 0;  // pairs with equal block read the same Q/K/V rows (cp_attn_plan)
 };
 
 cp_status run_pairs(const void* q, const void* k, const void* v, int64_t q_rows, int64_t k_rows, int hq, int hkv,
@@ -156,13 +159,19 @@ cp_status run_pairs(const void* q, const void* k, const void* v, int64_t q_rows,
   uint32_t* err = nullptr;
   if ((s = err_word(&err)) != CP_OK) return s;
 
+  // Pairs of one block run together (stable: the heaviest-first order of the
+  // caller is kept inside each block).
+  std::vector<const PairIn*> order;
+  order.reserve(pairs.size());
+  for (const PairIn& pi : pairs) order.push_back(&pi);
+  std::stable_sort(order.begin(), order.end(), [](const PairIn* a, const PairIn* b) { return a->block < b->block; });
+
   static cp_attn_plan plan;  // large POD: keep it off the stack
   static std::mutex plan_mu;
   std::lock_guard<std::mutex> lk(plan_mu);
-  for (size_t base = 0; base < pairs.size(); base += CP_MAX_PAIRS) {
-    const size_t cnt = std::min(pairs.size() - base, (size_t)CP_MAX_PAIRS);
+  size_t i = 0;
+  while (i < order.size()) {
     memset(&plan, 0, sizeof(plan));
-    plan.n_pairs = (int)cnt;
     plan.hq = hq;
     plan.hkv = hkv;
     plan.causal = causal ? 1 : 0;
@@ -170,22 +179,38 @@ cp_status run_pairs(const void* q, const void* k, const void* v, int64_t q_rows,
     plan.cu_seqlens = cu_dev;
     plan.scale_log2 = scale * 1.4426950408889634f;
     plan.err = err;
-    int ctas = 0;
-    for (size_t i = 0; i < cnt; ++i) {
-      const PairIn& pi = pairs[base + i];
-      cp_pair_desc& d = plan.pairs[i];
+    int ctas = 0, qt = 0;
+    int cur_block = -1;
+    // fill one launch: at most CP_MAX_PAIRS pairs in at most CP_MAX_BLOCKS blocks
+    while (i < order.size() && plan.n_pairs < CP_MAX_PAIRS) {
+      const PairIn& pi = *order[i];
+      if (pi.block != cur_block) {
+        if (plan.n_blocks == CP_MAX_BLOCKS) break;
+        if (plan.n_blocks > 0) ctas += qt * hq;  // close the previous block
+        plan.blk_cta_begin[plan.n_blocks] = ctas;
+        plan.blk_pair_begin[plan.n_blocks] = plan.n_pairs;
+        ++plan.n_blocks;
+        cur_block = pi.block;
+        qt = 0;
+      }
+      cp_pair_desc& d = plan.pairs[plan.n_pairs++];
       d.nq = (int)pi.q.size();
       d.nk = (int)pi.k.size();
       for (int x = 0; x < d.nq; ++x) d.q[x] = {pi.q[x].buf_row, pi.q[x].pos, pi.q[x].len, pi.q[x].out_row};
       for (int x = 0; x < d.nk; ++x) d.k[x] = {pi.k[x].buf_row, pi.k[x].pos, pi.k[x].len, 0};
       d.qtiles = pi.qtiles;
-      d.cta_begin = ctas;
+      d.qt_begin = qt;
       d.reverse = pi.reverse ? 1 : 0;
       d.lse_ld = pi.lse_ld;
       d.o = pi.o;
       d.lse = pi.lse;
-      ctas += pi.qtiles * hq;
+      qt += pi.qtiles;
+      plan.blk_qtiles[plan.n_blocks - 1] = qt;
+      ++i;
     }
+    ctas += qt * hq;
+    plan.blk_cta_begin[plan.n_blocks] = ctas;
+    plan.blk_pair_begin[plan.n_blocks] = plan.n_pairs;
     plan.total_ctas = ctas;
     cudaError_t e = launch_attn(dh, tq, tk, tv, plan, st);
     if (e != cudaSuccess) return cuda_fail(e, "attention launch");
@@ -236,13 +261,14 @@ cp_status run_merge(const std::vector<MergeTaskIn>& tasks_in, int h, int dh, flo
   static cp_merge_plan plan;
   static std::mutex mu;
   std::lock_guard<std::mutex> lk(mu);
-  // Tasks with more partials per row first: CTAs start in task order, so the
-  // long ones do not form the tail of the launch.
+  // Tasks with more partials per row first: CTAs start in task order and a
+  // CTA's time grows with its task's partial count, so the slow CTAs do not
+  // form the tail of the launch.
   std::vector<const MergeTaskIn*> order;
   order.reserve(tasks_in.size());
   for (const MergeTaskIn& t : tasks_in) order.push_back(&t);
   std::stable_sort(order.begin(), order.end(), [](const MergeTaskIn* a, const MergeTaskIn* b) {
-    return (int64_t)a->in.size() * a->rows > (int64_t)b->in.size() * b->rows;
+    return a->in.size() > b->in.size();
   });
   std::vector<MergeTaskIn> tasks;
   tasks.reserve(order.size());
@@ -257,22 +283,26 @@ cp_status run_merge(const std::vector<MergeTaskIn>& tasks_in, int h, int dh, flo
     plan.o_out = o_out;
     plan.lse_out = lse_out;
     plan.o_out_bf16 = static_cast<uint16_t*>(o_bf16);
-    int n_in = 0, max_rows = 0;
+    int n_in = 0;
+    long long ctas = 0;
     while (i < tasks.size() && plan.n_tasks < CP_MAX_TASKS &&
            n_in + (int)tasks[i].in.size() <= CP_MAX_INPUTS) {
       const MergeTaskIn& t = tasks[i];
+      const long long task_ctas = merge_task_ctas(t.rows, h);
+      if (ctas + task_ctas > INT32_MAX) break;
       cp_merge_task& d = plan.tasks[plan.n_tasks++];
       d.out_row0 = t.out_row0;
       d.rows = t.rows;
       d.n_in = (int)t.in.size();
       d.in_begin = n_in;
       d.head_off = t.head_off;
+      d.cta_begin = (int)ctas;
       for (const Merge& m : t.in) plan.inputs[n_in++] = {m.o, m.lse, m.row0, m.lse_ld};
-      max_rows = std::max(max_rows, t.rows);
+      ctas += task_ctas;
       ++i;
     }
     if (plan.n_tasks == 0) return fail(CP_ERR_UNSUPPORTED, "merge task with more than %d inputs", CP_MAX_INPUTS);
-    cudaError_t e = launch_merge(plan, max_rows, st);
+    cudaError_t e = launch_merge(plan, (int)ctas, st);
     if (e != cudaSuccess) return cuda_fail(e, "merge launch");
   }
   return CP_OK;
@@ -598,6 +628,7 @@ cp_status cp_ulysses_attn_fwd(const void* q, const void* k, const void* v, int S
     pi.lse = lse + (ptrdiff_t)r * hg * S - (ptrdiff_t)r * S;
     pi.lse_ld = S;
     pi.reverse = mask == CP_MASK_CAUSAL;
+    pi.block = r;
     pairs.push_back(std::move(pi));
   }
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)dh);
@@ -681,8 +712,9 @@ cp_status cp_usp_attn_fwd(const void* q, const void* k, const void* v, int S, in
     return cuda_fail(e, "usp seq->head");
 
   // Ring across the groups for every head block: head block u's rows start
-  // at u*S in the head-major buffers.  Pairs keep the heaviest-first order of
-  // the ring plan, head blocks interleaved.
+  // at u*S in the head-major buffers.  Each head block is one block of the
+  // launch (its pairs read rows [u*S, (u+1)*S)); inside it the pairs keep the
+  // heaviest-first order of the ring plan.
   std::vector<PairIn> pairs;
   pairs.reserve(plan.pairs.size() * Pu);
   for (const PairPlan& pp : plan.pairs)
@@ -698,6 +730,7 @@ cp_status cp_usp_attn_fwd(const void* q, const void* k, const void* v, int S, in
       pi.lse = reinterpret_cast<float*>(pu + pp.lse_off);
       pi.lse_ld = pp.rows;
       pi.reverse = mask == CP_MASK_CAUSAL;
+      pi.block = u;
       pairs.push_back(std::move(pi));
     }
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)dh);

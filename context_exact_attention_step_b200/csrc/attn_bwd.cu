@@ -142,10 +142,15 @@ struct DqIter {
         tl = 0;
         continue;
       }
-      const int ka = s.pos + ((pl->striped && j > r) ? 1 : 0) + off;
+      const int shift = (pl->striped && j > r) ? 1 : 0;
+      const int ka = s.pos + shift + off;
       if (ka > vis_hi) {  // positions grow along a segment
         ++sg;
         tl = 0;
+        continue;
+      }
+      if (ka + 127 < vis_lo) {  // keys of earlier documents: jump to the first visible tile
+        tl = (vis_lo - s.pos - shift) / 128;
         continue;
       }
       ++tl;
@@ -574,6 +579,10 @@ struct KvIter {
       if (qa > hi0) {  // positions grow along a segment
         ++sg;
         tl = 0;
+        continue;
+      }
+      if (qa + 127 < lo0 + shift) {  // queries before the key (or its document): jump over them
+        tl = (lo0 + shift - s.pos) / 128;
         continue;
       }
       ++tl;

@@ -14,10 +14,14 @@
 //
 // CTA layout (384 threads, one CTA per SM):
 //   warp 0      TMA producer: Q tile once, then K/V tiles into a 4-stage ring
-//   warp 1      tcgen05.mma issuer (one thread) and TMEM owner
-//   warps 2-3   idle
-//   warps 4-7   softmax of query sub-tile 0 (rows 0-127; one row per thread)
-//   warps 8-11  softmax of query sub-tile 1 (rows 128-255)
+//               (the whole warp runs the loop, an elected lane issues copies)
+//   warp 1      tcgen05.mma issuer (whole warp converged, an elected lane
+//               issues each MMA and commit) and TMEM owner
+//   warps 2-3   no work: they complete the control warpgroup, whose four
+//               warps give back registers together (setmaxnreg)
+//   warps 4-7   softmax and epilogue of query sub-tile 0 (rows 0-127; one
+//               row per thread)
+//   warps 8-11  softmax and epilogue of query sub-tile 1 (rows 128-255)
 // TMEM (512 columns): S0 | S1 (128 fp32 columns each; P is written back over
 // S as packed bf16) | O0 | O1 (dh columns each).
 // Tensor-pipe order per key tile j: PV0(j), S0(j+1), PV1(j), S1(j+1), so
@@ -29,6 +33,7 @@
 #include <math_constants.h>
 
 #include <atomic>
+#include <climits>
 
 #include "plan.h"
 #include "sm100_ptx.cuh"
@@ -50,6 +55,10 @@ constexpr int kThreads = 384;
 #endif
 constexpr int kPolyEvery = CP_POLY_EVERY;
 constexpr int kLoNone = -(1 << 30);
+// Document tables with fewer entries than this are copied into shared memory
+// at CTA start, so the per-CTA and per-row document lookups (binary searches)
+// do not wait on global-memory latency.
+constexpr int kCuSmem = 1024;
 constexpr int kHiNone = (1 << 30);
 
 template <int DH>
@@ -60,7 +69,7 @@ struct AttnCfg {
   static constexpr int kStages = DH == 128 ? 4 : 8;
   static constexpr int kQBytes = 2 * kTileBytes;
   static constexpr int kBarBytes = 256;
-  static constexpr int kSmemBytes = 1024 + kQBytes + kStages * kTileBytes + kBarBytes;
+  static constexpr int kSmemBytes = 1024 + kQBytes + kStages * kTileBytes + kBarBytes + kCuSmem * 4;
   static constexpr uint32_t kTmemCols = 512;
   // TMEM column of the S/P tile and of the O accumulator of sub-tile t
   __device__ static constexpr uint32_t col_s(int t) { return (uint32_t)t * 128u; }
@@ -79,6 +88,7 @@ struct KIter {
   const cp_pair_desc* pd;
   int seg, t;
   int vis_lo[2], vis_hi[2];
+  int lo_min;  // first position visible to either live sub-tile
   bool alive[2];
 
   __device__ bool next(KTile& out) {
@@ -96,6 +106,13 @@ struct KIter {
       if ((!alive[0] || ka > vis_hi[0]) && (!alive[1] || ka > vis_hi[1])) {
         ++seg;
         t = 0;
+        continue;
+      }
+      // Tiles that end before both windows start (keys of earlier documents)
+      // are jumped over in one step, to the tile holding the first visible
+      // position.
+      if (ka + CP_KV_TILE - 1 < lo_min) {
+        t = (lo_min - pd->k[seg].pos) / CP_KV_TILE;
         continue;
       }
       ++t;
@@ -117,20 +134,22 @@ struct KIter {
 };
 
 // Index of the document holding position x (cu = prefix sums, n_docs docs).
-__device__ __forceinline__ int doc_index(const int32_t* __restrict__ cu, int n_docs, int x) {
+// cu is the CTA's shared-memory copy of the table, or the global table when
+// it is too long to copy (generic loads serve both).
+__device__ __forceinline__ int doc_index(const int32_t* cu, int n_docs, int x) {
   int lo = 0, hi = n_docs - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (__ldg(cu + mid) <= x) lo = mid; else hi = mid - 1;
+    if (cu[mid] <= x) lo = mid; else hi = mid - 1;
   }
   return lo;
 }
-__device__ __forceinline__ int doc_start(const int32_t* __restrict__ cu, int n_docs, int x) {
-  return __ldg(cu + doc_index(cu, n_docs, x));
+__device__ __forceinline__ int doc_start(const int32_t* cu, int n_docs, int x) {
+  return cu[doc_index(cu, n_docs, x)];
 }
 // Last position of the document holding x.
-__device__ __forceinline__ int doc_last(const int32_t* __restrict__ cu, int n_docs, int x) {
-  return __ldg(cu + doc_index(cu, n_docs, x) + 1) - 1;
+__device__ __forceinline__ int doc_last(const int32_t* cu, int n_docs, int x) {
+  return cu[doc_index(cu, n_docs, x) + 1] - 1;
 }
 
 struct Item {
@@ -142,16 +161,22 @@ struct Item {
   bool alive[2];
 };
 
-__device__ __forceinline__ void decode_item(const cp_attn_plan& plan, Item& it) {
+// CTA -> (block, head, pair, query tile): head-major inside each block.
+__device__ __forceinline__ void decode_item(const cp_attn_plan& plan, const int32_t* cu, Item& it) {
   const int cta = blockIdx.x;
-  int p = 0;
-  while (p + 1 < plan.n_pairs && plan.pairs[p + 1].cta_begin <= cta) ++p;
+  int b = 0;
+  while (b + 1 < plan.n_blocks && plan.blk_cta_begin[b + 1] <= cta) ++b;
+  const int local = cta - plan.blk_cta_begin[b];
+  const int nqt = plan.blk_qtiles[b];
+  it.h = local / nqt;
+  int qt = local - it.h * nqt;
+  int p = plan.blk_pair_begin[b];
+  const int p_end = plan.blk_pair_begin[b + 1];
+  while (p + 1 < p_end && plan.pairs[p + 1].qt_begin <= qt) ++p;
   const cp_pair_desc* pd = &plan.pairs[p];
-  const int local = cta - pd->cta_begin;
+  qt -= pd->qt_begin;
   it.pd = pd;
-  it.h = local / pd->qtiles;
   it.hk = it.h / (plan.hq / plan.hkv);
-  int qt = local - it.h * pd->qtiles;
   if (pd->reverse) qt = pd->qtiles - 1 - qt;
   int s = 0;
   for (; s < pd->nq; ++s) {
@@ -170,11 +195,11 @@ __device__ __forceinline__ void decode_item(const cp_attn_plan& plan, Item& it) 
     const int qa = it.q_pos0 + t * 128;
     const int qb = qa + max(vt, 1) - 1;
     const bool varlen = plan.n_docs > 0;
-    it.vis_lo[t] = varlen ? doc_start(plan.cu_seqlens, plan.n_docs, qa) : kLoNone;
-    it.full_lo[t] = varlen ? doc_start(plan.cu_seqlens, plan.n_docs, qb) : kLoNone;
+    it.vis_lo[t] = varlen ? doc_start(cu, plan.n_docs, qa) : kLoNone;
+    it.full_lo[t] = varlen ? doc_start(cu, plan.n_docs, qb) : kLoNone;
     // upper key limit of a row: itself (causal) or its document's end
-    it.vis_hi[t] = plan.causal ? qb : (varlen ? doc_last(plan.cu_seqlens, plan.n_docs, qb) : kHiNone);
-    it.full_hi[t] = plan.causal ? qa : (varlen ? doc_last(plan.cu_seqlens, plan.n_docs, qa) : kHiNone);
+    it.vis_hi[t] = plan.causal ? qb : (varlen ? doc_last(cu, plan.n_docs, qb) : kHiNone);
+    it.full_hi[t] = plan.causal ? qa : (varlen ? doc_last(cu, plan.n_docs, qa) : kHiNone);
   }
 }
 
@@ -187,6 +212,7 @@ __device__ __forceinline__ void make_iter(const Item& it, KIter& ki) {
     ki.vis_hi[t] = it.vis_hi[t];
     ki.alive[t] = it.alive[t];
   }
+  ki.lo_min = min(it.alive[0] ? it.vis_lo[0] : INT_MAX, it.alive[1] ? it.vis_lo[1] : INT_MAX);
 }
 
 template <int DH>
@@ -204,11 +230,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             B_O = B_P + 4, B_DRAIN = B_O + 2, B_COUNT = B_DRAIN + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + B_COUNT);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  int32_t* s_cu = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(bars) + C::kBarBytes);
   auto bar = [&](int i) { return smem_addr(bars + i); };
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   uint32_t* err = plan.err;
+  const int32_t* cu = plan.cu_seqlens;
+  if (plan.n_docs > 0 && plan.n_docs < kCuSmem) {
+    for (int i = threadIdx.x; i <= plan.n_docs; i += kThreads) s_cu[i] = __ldg(plan.cu_seqlens + i);
+    cu = s_cu;  // read after the __syncthreads below
+  }
 
   if (threadIdx.x == 0) {
     mbar_init(bar(B_Q), 1);
@@ -241,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_holder;
 
   Item it;
-  decode_item(plan, it);
+  decode_item(plan, cu, it);
 
   // Registers: launched at 168 per thread (384 threads); inside its own
   // branch the control warpgroup (warps 0-3) drops to 56 and the two softmax
@@ -385,9 +417,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool rvalid = grow < it.q_valid;
     const int qpos = it.q_pos0 + grow;
     const bool varlen = plan.n_docs > 0;
-    const int row_lo = rvalid ? (varlen ? doc_start(plan.cu_seqlens, plan.n_docs, qpos) : kLoNone) : kHiNone;
+    const int row_lo = rvalid ? (varlen ? doc_start(cu, plan.n_docs, qpos) : kLoNone) : kHiNone;
     const int row_hi =
-        rvalid ? (plan.causal ? qpos : (varlen ? doc_last(plan.cu_seqlens, plan.n_docs, qpos) : kHiNone)) : kLoNone;
+        rvalid ? (plan.causal ? qpos : (varlen ? doc_last(cu, plan.n_docs, qpos) : kHiNone)) : kLoNone;
     const float scale_log2 = plan.scale_log2;
     const int full_lo = t == 0 ? it.full_lo[0] : it.full_lo[1];
     const int full_hi = t == 0 ? it.full_hi[0] : it.full_hi[1];
@@ -535,32 +567,49 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok) {
       tc_fence_after();
+      // Epilogue.  O leaves TMEM one row per thread; stored from there, one
+      // warp instruction would touch 32 rows 16 KB apart.  Instead each
+      // 32-column slab goes through a 4 KB shared-memory tile per warp (in the
+      // K/V stage buffers, idle once every MMA has completed), 16-byte chunks
+      // XOR-swizzled by row so that both the row-wise writes and the
+      // column-wise reads take the minimum of four wavefronts, and leaves as
+      // four whole 128-byte row segments per store instruction.
       const cp_pair_desc* pd = it.pd;
       const int orow = it.out_row0 + grow;
-      float* op = pd->o + ((size_t)orow * plan.hq + it.h) * DH;
       const float inv_l = l > 0.f ? pend / l : 0.f;
-      if (n_tiles > 0) {
+      float4* stile = reinterpret_cast<float4*>(sKV + (warp - 4) * 4096);
+      const int wrow0 = t * 128 + quarter * 32;  // CTA row of lane 0 of this warp
+      const int cc = lane & 7;
+      fence_proxy_async_smem();
 #pragma unroll 1
-        for (int ch = 0; ch < DH / 32; ++ch) {
-          uint32_t o[32];
+      for (int ch = 0; ch < DH / 32; ++ch) {
+        uint32_t o[32];
+        if (n_tiles > 0) {
           tmem_ld32(tO + ch * 32, o);
           tc_wait_ld();
-          if (rvalid) {
-            float4* dst = reinterpret_cast<float4*>(op + ch * 32);
+        }
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              float4 v;
-              v.x = l > 0.f ? __uint_as_float(o[4 * i + 0]) * inv_l : 0.f;
-              v.y = l > 0.f ? __uint_as_float(o[4 * i + 1]) * inv_l : 0.f;
-              v.z = l > 0.f ? __uint_as_float(o[4 * i + 2]) * inv_l : 0.f;
-              v.w = l > 0.f ? __uint_as_float(o[4 * i + 3]) * inv_l : 0.f;
-              dst[i] = v;
-            }
+        for (int c = 0; c < 8; ++c) {
+          float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (n_tiles > 0 && l > 0.f) {
+            v.x = __uint_as_float(o[4 * c + 0]) * inv_l;
+            v.y = __uint_as_float(o[4 * c + 1]) * inv_l;
+            v.z = __uint_as_float(o[4 * c + 2]) * inv_l;
+            v.w = __uint_as_float(o[4 * c + 3]) * inv_l;
+          }
+          stile[lane * 8 + (c ^ (lane & 7))] = v;
+        }
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int rr = 4 * i + (lane >> 3);  // lanes 8k..8k+7 write one row's 128 bytes
+          const float4 v = stile[rr * 8 + (cc ^ (rr & 7))];
+          if (wrow0 + rr < it.q_valid) {
+            float* dst = pd->o + ((size_t)(it.out_row0 + wrow0 + rr) * plan.hq + it.h) * DH + ch * 32;
+            reinterpret_cast<float4*>(dst)[cc] = v;
           }
         }
-      } else if (rvalid) {
-        float4* dst = reinterpret_cast<float4*>(op);
-        for (int i = 0; i < DH / 4; ++i) dst[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        __syncwarp();
       }
       if (rvalid) {
         const float lse = l > 0.f ? (m_used + __log2f(l)) * 0.69314718055994531f : -CUDART_INF_F;

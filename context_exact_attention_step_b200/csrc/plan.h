@@ -8,8 +8,9 @@
 
 #define CP_MAX_SEGS 4        // row segments per side of one block pair
 #define CP_MAX_PAIRS 64      // block pairs per attention launch
-#define CP_MAX_TASKS 32      // merge tasks per merge launch
-#define CP_MAX_INPUTS 192    // merge inputs per merge launch
+#define CP_MAX_BLOCKS 16     // pair blocks per attention launch (see cp_attn_plan)
+#define CP_MAX_TASKS 128     // merge tasks per merge launch
+#define CP_MAX_INPUTS 512    // merge inputs per merge launch
 #define CP_Q_TILE 256        // query rows per CTA (two 128-row MMA tiles)
 #define CP_KV_TILE 128       // key/value rows per pipeline stage (and per S tile)
 
@@ -31,16 +32,26 @@ struct cp_pair_desc {
   cp_seg q[CP_MAX_SEGS];
   cp_seg k[CP_MAX_SEGS];
   int32_t qtiles;     // sum over q segments of ceil(len / CP_Q_TILE)
-  int32_t cta_begin;  // first CTA of this pair in the launch
+  int32_t qt_begin;   // first query tile of this pair among its block's tiles of one head
   int32_t reverse;    // visit the query tiles last-first (heaviest first under causal)
   int32_t lse_ld;     // row pitch of the LSE output ([hq][lse_ld])
   float* o;           // O output, [rows][hq][dh] fp32
   float* lse;         // LSE output, [hq][lse_ld] fp32
 };
 
+// The pairs of a launch come in blocks: the pairs of one block read the same
+// Q/K/V rows (all ring steps of one ring), different blocks read different
+// rows (the head groups of Ulysses, the head blocks of the hybrid).  Inside a
+// block the CTAs run head-major -- every query tile of every pair of head 0,
+// then head 1, ... -- so the CTAs resident at one time share one head's Q and
+// K/V through L2 instead of streaming every head's side by side.
 struct cp_attn_plan {
   int32_t n_pairs;
   int32_t total_ctas;
+  int32_t n_blocks;
+  int32_t blk_cta_begin[CP_MAX_BLOCKS + 1];   // CTAs of block b: [blk_cta_begin[b], blk_cta_begin[b + 1])
+  int32_t blk_pair_begin[CP_MAX_BLOCKS + 1];  // pairs of block b: [blk_pair_begin[b], blk_pair_begin[b + 1])
+  int32_t blk_qtiles[CP_MAX_BLOCKS];          // query tiles per head of block b
   int32_t hq, hkv;
   int32_t causal;
   int32_t n_docs;               // 0: no document mask
@@ -68,6 +79,7 @@ struct cp_merge_task {
   int32_t n_in;
   int32_t in_begin;
   int32_t head_off;      // first output head of the task's h heads
+  int32_t cta_begin;     // first CTA of the task in the launch (tasks in CTA order)
 };
 
 struct cp_merge_plan {

@@ -330,6 +330,13 @@ __device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x) {
   return f2_pack(r0, r1);
 }
 
+// Orders this thread's generic-proxy shared-memory accesses with later
+// async-proxy ones (TMA, tcgen05) and earlier async-proxy writes with later
+// generic reads of the same bytes.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

@@ -45,15 +45,6 @@ std::atomic<uint64_t>& launch_counter();
 __device__ uint32_t g_attn_err = 0;
 
 constexpr int kThreads = 384;
-// Every kPolyEvery-th column pair of an unmasked tile takes the software
-// exp2 on the FMA pipe instead of MUFU (0 disables it).  Measured on B200 the
-// softmax is bound by instruction latency rather than MUFU throughput, and
-// the longer instruction stream of the software path made every tested
-// fraction (1/4, 1/3, 1/2) slower, so it is off by default.
-#ifndef CP_POLY_EVERY
-#define CP_POLY_EVERY 0
-#endif
-constexpr int kPolyEvery = CP_POLY_EVERY;
 constexpr int kLoNone = -(1 << 30);
 // Document tables with fewer entries than this are copied into shared memory
 // at CTA start, so the per-CTA and per-row document lookups (binary searches)
@@ -164,15 +155,20 @@ struct Item {
 // CTA -> (block, head, pair, query tile): head-major inside each block.
 __device__ __forceinline__ void decode_item(const cp_attn_plan& plan, const int32_t* cu, Item& it) {
   const int cta = blockIdx.x;
-  int b = 0;
+  int b = 0;  // at most CP_MAX_BLOCKS entries, adjacent in the parameter block
   while (b + 1 < plan.n_blocks && plan.blk_cta_begin[b + 1] <= cta) ++b;
   const int local = cta - plan.blk_cta_begin[b];
   const int nqt = plan.blk_qtiles[b];
   it.h = local / nqt;
   int qt = local - it.h * nqt;
+  // the last pair of the block whose first tile is <= qt (binary search: a
+  // linear scan would touch a new line of the parameter block per pair)
   int p = plan.blk_pair_begin[b];
-  const int p_end = plan.blk_pair_begin[b + 1];
-  while (p + 1 < p_end && plan.pairs[p + 1].qt_begin <= qt) ++p;
+  int p_hi = plan.blk_pair_begin[b + 1] - 1;
+  while (p < p_hi) {
+    const int mid = (p + p_hi + 1) >> 1;
+    if (plan.pairs[mid].qt_begin <= qt) p = mid; else p_hi = mid - 1;
+  }
   const cp_pair_desc* pd = &plan.pairs[p];
   qt -= pd->qt_begin;
   it.pd = pd;
@@ -276,10 +272,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   decode_item(plan, cu, it);
 
   // Registers: launched at 168 per thread (384 threads); inside its own
-  // branch the control warpgroup (warps 0-3) drops to 56 and the two softmax
-  // warpgroups rise to 216: 128 * 56 + 256 * 216 = 62464 <= 384 * 168 = 64512.
+  // branch the control warpgroup (warps 0-3) drops to 80 and the two softmax
+  // warpgroups rise to 192: 128 * 80 + 256 * 192 = 59392 <= 384 * 168 = 64512.
   if (warp < 4) {
-    regs_dec<56>();
+    regs_dec<80>();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -405,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_wait_warp(bar(B_DRAIN), 0, abort_flag, nullptr, 1000000000ull);
   }
   } else {
-    regs_inc<216>();
+    regs_inc<192>();
     // ------------------------------------------------------------ softmax
     const int t = (warp - 4) >> 2;
     const int quarter = warp & 3;
@@ -462,13 +458,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
       tc_wait_ld();
       const bool full = kt.valid == CP_KV_TILE && kt.pos >= full_lo && kt.pos + CP_KV_TILE - 1 <= full_hi;
-      if (!full) {
-        const int clo = row_lo - kt.pos;
-        const int chi = min(row_hi - kt.pos, kt.valid - 1);
+      const int clo = row_lo - kt.pos;
+      const int chi = min(row_hi - kt.pos, kt.valid - 1);
+      // -inf outside this row's visible keys, for columns [c0, c1)
+      auto mask_cols = [&](int c0, int c1) {
 #pragma unroll
         for (int c = 0; c < 128; ++c)
-          if (c < clo || c > chi) s[c] = __float_as_uint(-CUDART_INF_F);
-      }
+          if (c >= c0 && c < c1 && (c < clo || c > chi)) s[c] = __float_as_uint(-CUDART_INF_F);
+      };
+      if (!full) mask_cols(0, 128);
       // S(j) is complete, hence so is PV(j-1): apply a pending rescale of O
       // before P(j) is released.
       if (__any_sync(0xffffffffu, pend != 1.f)) {
@@ -489,41 +487,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       uint32_t pk[32];
       uint64_t lsum = f2_pack(0.f, 0.f);
-      // P = 2^(x - ref) for columns [64h, 64h + 64), packed to bf16 pairs.
-      // On tiles without masked entries every kPolyEvery-th column pair uses
-      // the FMA-pipe exp2 so that the MUFU unit is not the bottleneck.
-      auto exp_half = [&](int h) {
+      float ma = -CUDART_INF_F;
+      // P = 2^(x - ref) for columns [64h, 64h + 64), packed to bf16 pairs;
+      // with fold_max the maximum of those columns is taken on the way, so
+      // each score register dies as soon as its exponential is formed.
+      auto exp_half = [&](int h, bool fold_max) {
         const float nr = ref == -CUDART_INF_F ? 0.f : -ref;
         const uint64_t nr2 = f2_pack(nr, nr);
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
-          const uint64_t x = f2_fma(f2_pack(__uint_as_float(s[h * 64 + 2 * c]), __uint_as_float(s[h * 64 + 2 * c + 1])),
-                                    c2, nr2);
-          float p0, p1;
-          if (kPolyEvery > 0 && (c % kPolyEvery) == kPolyEvery - 1 && full) {
-            f2_unpack(exp2_poly_x2(x), p0, p1);
-          } else {
-            float x0, x1;
-            f2_unpack(x, x0, x1);
-            p0 = ex2_approx(x0);
-            p1 = ex2_approx(x1);
-          }
+          const float s0 = __uint_as_float(s[h * 64 + 2 * c]), s1 = __uint_as_float(s[h * 64 + 2 * c + 1]);
+          if (fold_max) ma = max3f(ma, s0, s1);
+          const uint64_t x = f2_fma(f2_pack(s0, s1), c2, nr2);
+          float x0, x1;
+          f2_unpack(x, x0, x1);
+          const float p0 = ex2_approx(x0);
+          const float p1 = ex2_approx(x1);
           lsum = f2_add(lsum, f2_pack(p0, p1));
           pk[c] = pack_bf16x2(p0, p1);
         }
       };
-      exp_half(0);
+      exp_half(0, true);
       // Tile maximum, checked before the first half of P is released.
-      float ma = -CUDART_INF_F, mb = -CUDART_INF_F;
+      float mb = -CUDART_INF_F, mc = -CUDART_INF_F;
 #pragma unroll
-      for (int c = 0; c < 128; c += 4) {
-        ma = max3f(ma, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
-        mb = max3f(mb, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
+      for (int c = 64; c < 128; c += 4) {
+        mb = max3f(mb, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+        mc = max3f(mc, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
       }
-      const float mt = fmaxf(ma, mb) * scale_log2;
+      const float mt = fmaxf(ma, fmaxf(mb, mc)) * scale_log2;
       // Guard: P must stay far from the bf16 / fp32 range limits.  A row whose
       // tile maximum exceeds the reference by more than 2^64 re-bases now
-      // (rescaling what O and l hold) and recomputes its P.
+      // (rescaling what O and l hold) and recomputes its P; the first half of
+      // the scores is read again from TMEM, where P has not yet replaced it.
       const bool over = mt > ref + 64.f;
       if (__any_sync(0xffffffffu, over)) {
         float f = 1.f;
@@ -533,15 +529,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           l *= f;
         }
         if (n_tiles > 0) rescale_o(f);
+        tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+        tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+        tc_wait_ld();
+        if (!full) mask_cols(0, 64);
         lsum = f2_pack(0.f, 0.f);
-        exp_half(0);
+        exp_half(0, false);
       }
       tmem_st32(tS + 0, pk);
       tc_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(B_P + 2 * t + 0));
-      exp_half(1);
+      exp_half(1, false);
       tmem_st32(tS + 32, pk);
       tc_wait_st();
       tc_fence_before();

@@ -302,34 +302,6 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return d;
 }
 
-// Software 2^x for two lanes on the FMA pipe (no MUFU), relative error
-// <= 7.5e-5, for x in [-125, 64] (inputs below -125 give about 2^-125).
-// Cody-Waite range reduction 2^x = 2^n 2^f, n = round(x) obtained by adding
-// 1.5 * 2^23, f = x - n in [-1/2, 1/2]; 2^f from a degree-3 minimax
-// polynomial (coefficients from csrc/gen_exp2_poly.py, Remez exchange);
-// 2^n enters by an integer add to the exponent field.
-__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x) {
-  float x0, x1;
-  f2_unpack(x, x0, x1);
-  x0 = fmaxf(x0, -125.f);
-  x1 = fmaxf(x1, -125.f);
-  const uint64_t xc = f2_pack(x0, x1);
-  const uint64_t t = f2_add(xc, f2_pack(12582912.f, 12582912.f));     // 1.5 * 2^23 + round(x)
-  const uint64_t n = f2_add(t, f2_pack(-12582912.f, -12582912.f));    // round(x)
-  const uint64_t f = f2_fma(n, f2_pack(-1.f, -1.f), xc);               // x - round(x)
-  uint64_t p = f2_fma(f, f2_pack(5.517166853e-02f, 5.517166853e-02f), f2_pack(2.426111251e-01f, 2.426111251e-01f));
-  p = f2_fma(p, f, f2_pack(6.932609677e-01f, 6.932609677e-01f));
-  p = f2_fma(p, f, f2_pack(9.999280572e-01f, 9.999280572e-01f));
-  float p0, p1, t0, t1;
-  f2_unpack(p, p0, p1);
-  f2_unpack(t, t0, t1);
-  // the low bits of t hold round(x) in two's complement; shifting them into
-  // the exponent field multiplies by 2^round(x)
-  const float r0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
-  const float r1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
-  return f2_pack(r0, r1);
-}
-
 // Orders this thread's generic-proxy shared-memory accesses with later
 // async-proxy ones (TMA, tcgen05) and earlier async-proxy writes with later
 // generic reads of the same bytes.

@@ -67,6 +67,12 @@ BWD_SUITE = ["ring_contig_32k", "varlen_zigzag_128k"]
 # change makes the entry stale and the line reports null until the capture is
 # repeated.  Filled from the profiles/ summaries.
 ATTN_TRAFFIC = {
+    # profiles/attn_fwd_kernel_dram_ring_workloads.md (one-pass DRAM read + write per launch)
+    ("0f2224ea9ddfd474", "ring_contig_32k"): 2.1437e9,
+    ("0f2224ea9ddfd474", "ring_zigzag_64k"): 9.7940e9,
+    ("0f2224ea9ddfd474", "varlen_zigzag_128k"): 9.9621e9,
+    ("0f2224ea9ddfd474", "ring_striped_64k"): 13.6606e9,
+    ("0f2224ea9ddfd474", "ulysses_gqa_128k"): 6.7052e9,
 }
 
 
@@ -219,6 +225,7 @@ def make_workload(name, seq_len=None, pass_="fwd", host=False):
     K, V; after: the inverse reorder of O and LSE)."""
     from context_exact_attention_step_b200 import api, synth
     cfg = dict(synth.CONFIGS[name])
+    resized = bool(seq_len) and int(seq_len) != cfg["S"]
     if seq_len:
         cfg["S"] = int(seq_len)
     S, hq, hkv, dh, P = cfg["S"], cfg["hq"], cfg["hkv"], cfg["dh"], cfg["P"]
@@ -229,7 +236,7 @@ def make_workload(name, seq_len=None, pass_="fwd", host=False):
         cu = synth.cu_seqlens_from_lengths(synth.doc_lengths(S, cfg["doc_lo"], cfg["doc_hi"])).tolist()
     layout = cfg["layout"]
     dev = torch.device("cuda")
-    w = dict(name=name, cfg=cfg, S=S, hq=hq, hkv=hkv, dh=dh, P=P, layout=layout, cu=cu, dtype=dtype)
+    w = dict(name=name, cfg=cfg, S=S, hq=hq, hkv=hkv, dh=dh, P=P, layout=layout, cu=cu, dtype=dtype, resized=resized)
     w["pairs"] = api.count_live_pairs(S, True, cu)
     w["flops"] = 4.0 * dh * hq * w["pairs"]
     if host:
@@ -424,7 +431,8 @@ def summarize(w, r, pk, ws):
         return out
     out["attn"] = {"ms": am, "tflops": tflops(w["flops"], am), "frac": tflops(w["flops"], am) / pk["bf16"],
                    "frac_of_sustained": tflops(w["flops"], am) / pk["bf16_sus"],
-                   "traffic": ATTN_TRAFFIC.get((attn_src_hash(), w["name"]))}
+                   # the capture is of the full-size workload: none for a --seq-len override
+                   "traffic": ATTN_TRAFFIC.get((attn_src_hash(), w["name"])) if not w.get("resized") else None}
     if "merge" in r:
         mb = merge_bytes(w)
         mm = max_over_ranks(statistics.mean(r["merge"]), ws)

@@ -99,6 +99,49 @@ __device__ __forceinline__ void decode_own(const cp_bwd_plan& pl, uint32_t item,
   o.valid = min(128, s.len - tile * 128);
 }
 
+// One warp stores 32 rows (row = lane) x 32 fp32 columns, o[] * f (zeros when
+// `zero`): the values pass through the warp's 4 KB shared tile, 16-byte chunks
+// XOR-swizzled by row so that the row-wise writes and the column-wise reads
+// both take the minimum of four wavefronts, and leave as four whole 128-byte
+// row segments per store instruction (stored straight from the TMEM layout,
+// one warp instruction would touch 32 rows far apart).  Row r goes to
+// dst_row0 + r * pitch; rows >= n_rows are skipped; with accumulate the
+// destination is read and added.
+__device__ __forceinline__ void warp_store_32x32(float4* stile, const uint32_t (&o)[32], float f, bool zero,
+                                                 float* dst_row0, size_t pitch, int n_rows, bool accumulate) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (!zero) {
+      v.x = __uint_as_float(o[4 * c + 0]) * f;
+      v.y = __uint_as_float(o[4 * c + 1]) * f;
+      v.z = __uint_as_float(o[4 * c + 2]) * f;
+      v.w = __uint_as_float(o[4 * c + 3]) * f;
+    }
+    stile[lane * 8 + (c ^ (lane & 7))] = v;
+  }
+  __syncwarp();
+  const int cc = lane & 7;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int rr = 4 * i + (lane >> 3);  // lanes 8k..8k+7 take one row's 128 bytes
+    float4 v = stile[rr * 8 + (cc ^ (rr & 7))];
+    if (rr < n_rows) {
+      float4* d = reinterpret_cast<float4*>(dst_row0 + (size_t)rr * pitch) + cc;
+      if (accumulate) {
+        const float4 a = *d;
+        v.x += a.x;
+        v.y += a.y;
+        v.z += a.z;
+        v.w += a.w;
+      }
+      *d = v;
+    }
+  }
+  __syncwarp();
+}
+
 // ------------------------------------------------------------------ dQ side
 struct KvTile {
   int buf_row, pos, valid;
@@ -477,10 +520,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
     }
     if (ok) {
-      // warpgroup hh writes dQ columns [hh DH/2, (hh + 1) DH/2)
+      // warpgroup hh writes dQ columns [hh DH/2, (hh + 1) DH/2), staged in
+      // the K/V stage buffers (idle once every MMA has completed)
       tc_fence_after();
-      const size_t orow = (size_t)(own.buf_row0 - own.grp_row0 + row);
-      float* dst = plan.dq + (orow * plan.out_hq + own.grp * plan.hq + h) * DH + hh * (DH / 2);
+      const size_t orow0 = (size_t)(own.buf_row0 - own.grp_row0 + quarter * 32);
+      const size_t pitch = (size_t)plan.out_hq * DH;
+      float* dst = plan.dq + orow0 * pitch + (size_t)(own.grp * plan.hq + h) * DH + hh * (DH / 2);
+      float4* stile = reinterpret_cast<float4*>(sKV + (warp - 4) * 4096);
+      fence_proxy_async_smem();
 #pragma unroll 1
       for (int ch = 0; ch < DH / 64; ++ch) {
         uint32_t o[32];
@@ -488,25 +535,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tmem_ld32(tmem + lane_base + C::kColQ + hh * (DH / 2) + ch * 32, o);
           tc_wait_ld();
         }
-        if (rvalid) {
-          float4* d4 = reinterpret_cast<float4*>(dst + ch * 32);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            float4 v;
-            v.x = j > 0 ? __uint_as_float(o[4 * i + 0]) * plan.scale : 0.f;
-            v.y = j > 0 ? __uint_as_float(o[4 * i + 1]) * plan.scale : 0.f;
-            v.z = j > 0 ? __uint_as_float(o[4 * i + 2]) * plan.scale : 0.f;
-            v.w = j > 0 ? __uint_as_float(o[4 * i + 3]) * plan.scale : 0.f;
-            if (plan.accumulate) {
-              const float4 a = d4[i];
-              v.x += a.x;
-              v.y += a.y;
-              v.z += a.z;
-              v.w += a.w;
-            }
-            d4[i] = v;
-          }
-        }
+        warp_store_32x32(stile, o, plan.scale, j == 0, dst + ch * 32, pitch, own.valid - quarter * 32,
+                         plan.accumulate != 0);
       }
     }
   }
@@ -927,12 +957,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
     }
     if (ok) {
-      // warpgroup 0 writes dV, warpgroup 1 writes dK * scale
+      // warpgroup 0 writes dV, warpgroup 1 writes dK * scale, staged in the
+      // Q/dO stage buffers (idle once every MMA has completed)
       tc_fence_after();
-      const size_t orow = (size_t)(own.buf_row0 - own.grp_row0 + row) * plan.out_hkv + own.grp * plan.hkv + hk;
-      float* dst = (hh == 0 ? plan.dv : plan.dk) + orow * DH;
+      const size_t pitch = (size_t)plan.out_hkv * DH;
+      const size_t orow0 = (size_t)(own.buf_row0 - own.grp_row0 + quarter * 32);
+      float* dst = (hh == 0 ? plan.dv : plan.dk) + orow0 * pitch + (size_t)(own.grp * plan.hkv + hk) * DH;
       const uint32_t col = hh == 0 ? C::kColDV : C::kColDK;
       const float f = hh == 0 ? 1.f : plan.scale;
+      float4* stile = reinterpret_cast<float4*>(sStage + (warp - 4) * 4096);
+      fence_proxy_async_smem();
 #pragma unroll 1
       for (int ch = 0; ch < DH / 32; ++ch) {
         uint32_t o[32];
@@ -940,25 +974,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tmem_ld32(tmem + lane_base + col + ch * 32, o);
           tc_wait_ld();
         }
-        if (rvalid) {
-          float4* d4 = reinterpret_cast<float4*>(dst + ch * 32);
-#pragma unroll
-          for (int k4 = 0; k4 < 8; ++k4) {
-            float4 v;
-            v.x = i > 0 ? __uint_as_float(o[4 * k4 + 0]) * f : 0.f;
-            v.y = i > 0 ? __uint_as_float(o[4 * k4 + 1]) * f : 0.f;
-            v.z = i > 0 ? __uint_as_float(o[4 * k4 + 2]) * f : 0.f;
-            v.w = i > 0 ? __uint_as_float(o[4 * k4 + 3]) * f : 0.f;
-            if (plan.accumulate) {
-              const float4 a = d4[k4];
-              v.x += a.x;
-              v.y += a.y;
-              v.z += a.z;
-              v.w += a.w;
-            }
-            d4[k4] = v;
-          }
-        }
+        warp_store_32x32(stile, o, f, i == 0, dst + ch * 32, pitch, own.valid - quarter * 32, plan.accumulate != 0);
       }
     }
   }

@@ -9,10 +9,10 @@
 // denominator.  Partials whose LSE_i is -inf hold no admitted key for that row;
 // they get weight 0 and their O is never combined.  All arithmetic is fp32.
 //
-// A CTA takes a block of 8 rows x 8 heads of one task.  Its LSE inputs (8
-// consecutive rows of each head, one sector per head and partial) are staged
-// in shared memory first; then warp w folds row w, two (row, head) items at a
-// time with all their loads issued together:
+// A CTA takes a block of 8 rows x 8 heads of one task; warp w folds row w,
+// two (row, head) items at a time with all their loads (LSE and O of two
+// partials each) issued together, the 8 warps' LSE loads of one head and
+// partial falling in one sector:
 // dh/4 threads per (row, head), each owning four consecutive columns moved
 // with 16-byte loads and stores, so a warp instruction covers 512 contiguous
 // bytes of a row (dh = 128) and a warp's eight heads cover 4 KB.  The tasks of
@@ -32,14 +32,12 @@ std::atomic<uint64_t>& launch_counter();
 
 constexpr int kMergeRows = 8;    // rows per CTA (one per warp)
 constexpr int kMergeHeads = 8;   // heads per CTA
-constexpr int kMergeStaged = 16; // partials per task whose LSEs are staged in shared memory
 
 template <int DH>
 __global__ void __launch_bounds__(256, 5) lse_merge_kernel(const __grid_constant__ cp_merge_plan plan) {
   constexpr int TPI = DH / 4;     // threads per (row, head)
   constexpr int IPW = 32 / TPI;   // (row, head) items per warp instruction
   constexpr int U = 2;            // partials per item whose loads are in flight together
-  __shared__ float s_lse[kMergeStaged][kMergeHeads][kMergeRows];
   __shared__ float s_out[kMergeHeads][kMergeRows];
 
   const int cta = blockIdx.x;
@@ -57,21 +55,6 @@ __global__ void __launch_bounds__(256, 5) lse_merge_kernel(const __grid_constant
   const int h0 = (local - rb * n_hb) * kMergeHeads;
   const cp_merge_input* in = plan.inputs + task.in_begin;
   const int n = task.n_in;
-  const bool staged = n <= kMergeStaged;
-
-  if (staged) {
-    for (int e = threadIdx.x; e < n * kMergeHeads * kMergeRows; e += blockDim.x) {
-      const int i = e / (kMergeHeads * kMergeRows);
-      const int hh = (e / kMergeRows) % kMergeHeads;
-      const int rr = e % kMergeRows;
-      const int row = row0 + rr, head = h0 + hh;
-      float v = -CUDART_INF_F;
-      if (row < task.rows && head < h) v = __ldg(in[i].lse + (size_t)head * in[i].lse_ld + in[i].row0 + row);
-      s_lse[i][hh][rr] = v;
-    }
-    __syncthreads();
-  }
-
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int sub = lane % TPI;
@@ -104,8 +87,8 @@ __global__ void __launch_bounds__(256, 5) lse_merge_kernel(const __grid_constant
             o[a][u] = make_float4(0.f, 0.f, 0.f, 0.f);
             if (head[a] < h && i0 + u < n) {
               const cp_merge_input& x = in[i0 + u];
-              li[a][u] = staged ? s_lse[i0 + u][hh[a]][warp]
-                                : __ldg(x.lse + (size_t)head[a] * x.lse_ld + x.row0 + row);
+              // the 8 warps read 8 consecutive rows of this head: one sector
+              li[a][u] = __ldg(x.lse + (size_t)head[a] * x.lse_ld + x.row0 + row);
               o[a][u] = __ldcs(reinterpret_cast<const float4*>(x.o + ((size_t)(x.row0 + row) * h + head[a]) * DH) + sub);
             }
           }

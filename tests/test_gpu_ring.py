@@ -62,6 +62,21 @@ def test_varlen_zigzag_small():
     ring_case(S, 2, 2, 128, P, "zigzag", cu=cu)
 
 
+@pytest.mark.parametrize("n_docs", [300, 1100])
+def test_varlen_many_short_documents(n_docs):
+    """Many short documents (random cuts): most block pairs admit nothing
+    and the live ones are trimmed to a few rows at shard edges, every key
+    tile holds several documents, and with 1100 documents the document table
+    is too long for the attention kernel's shared-memory copy, so the kernel
+    reads it from global memory."""
+    S, P = 8192, 4
+    rng = np.random.default_rng(n_docs)
+    cuts = np.sort(rng.choice(np.arange(1, S), size=n_docs - 1, replace=False))
+    cu = [0] + cuts.tolist() + [S]
+    ring_case(S, 2, 2, 64, P, "zigzag", cu=cu)
+    ring_case(S, 2, 2, 64, P, "contiguous", cu=cu)
+
+
 def test_seq_equals_cp_size():
     # the pages' mask check: one token per rank
     ring_case(8, 2, 2, 64, 8, "contiguous")

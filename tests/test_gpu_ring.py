@@ -77,6 +77,17 @@ def test_varlen_many_short_documents(n_docs):
     ring_case(S, 2, 2, 64, P, "contiguous", cu=cu)
 
 
+def test_varlen_sixteen_ranks_many_documents():
+    """Sixteen zigzag ranks over 1100 short documents: 43 of the 256 block
+    pairs are live, each trimmed to the few rows whose documents cross a
+    chunk edge, so every rank's rows are cut into many merge tasks with
+    different sets of partials."""
+    S, P, n_docs = 16384, 16, 1100
+    rng = np.random.default_rng(7)
+    cuts = np.sort(rng.choice(np.arange(1, S), size=n_docs - 1, replace=False))
+    ring_case(S, 2, 2, 64, P, "zigzag", cu=[0] + cuts.tolist() + [S])
+
+
 def test_seq_equals_cp_size():
     # the pages' mask check: one token per rank
     ring_case(8, 2, 2, 64, 8, "contiguous")
@@ -90,6 +101,20 @@ def test_ulysses_small_gqa():
     torch.cuda.synchronize()
     want_o, want_l = ref.attention(f64(q), f64(k), f64(v), causal=True)
     compare(o, lse, want_o, want_l, what="ulysses")
+
+
+@pytest.mark.parametrize("P,hkv", [(16, 16), (32, 32)])
+def test_ulysses_many_head_groups(P, hkv):
+    # every head group is its own block of the attention launch: 16 blocks
+    # fill one launch, 32 need two (the plan is split at the block limit),
+    # CTAs head-major inside each block
+    S, hq, dh = 2048, 32, 64
+    q, k, v = synth.qkv(S, hq, hkv, dh, seeds=(31, 32, 33))
+    o, lse = api.ulysses_attn_fwd(q.cuda(), k.cuda(), v.cuda(), P)
+    torch.cuda.synchronize()
+    assert api.device_error() == 0
+    want_o, want_l = ref.attention(f64(q), f64(k), f64(v), causal=True)
+    compare(o, lse, want_o, want_l, what=f"ulysses P={P}")
 
 
 # ----------------------------------------------------------- full sizes

@@ -103,6 +103,23 @@ def test_ulysses_small_gqa():
     compare(o, lse, want_o, want_l, what="ulysses")
 
 
+def test_ring_and_ulysses_agree_at_fixed_length():
+    """The pages' A/B of Ring and Ulysses at one sequence length: both are
+    exact, so on the same inputs they give the same O and LSE (to the
+    kernels' rounding) and each matches the oracle."""
+    S, hq, hkv, dh, P = 4096, 8, 8, 128, 4
+    q, k, v = synth.qkv(S, hq, hkv, dh, seeds=(41, 42, 43))
+    qd, kd, vd = (t.cuda() for t in (q, k, v))
+    o_r, l_r = api.ring_attn_fwd(qd, kd, vd, P, "contiguous", True)
+    o_u, l_u = api.ulysses_attn_fwd(qd, kd, vd, P)
+    torch.cuda.synchronize()
+    assert api.device_error() == 0
+    want_o, want_l = ref.attention(f64(q), f64(k), f64(v), causal=True)
+    compare(o_r, l_r, want_o, want_l, what="ring")
+    compare(o_u, l_u, want_o, want_l, what="ulysses")
+    compare(o_r, l_r, f64(o_u), f64(l_u), what="ring vs ulysses")
+
+
 @pytest.mark.parametrize("P,hkv", [(16, 16), (32, 32)])
 def test_ulysses_many_head_groups(P, hkv):
     # every head group is its own block of the attention launch: 16 blocks

@@ -153,14 +153,38 @@ struct KvTile {
 struct DqIter {
   const cp_bwd_plan* pl;
   int r, t, sg, tl, row0;
+  int P, t_end;
+  bool striped;
+  // the current ring step's shard j = (r - t) mod P, its segment count and
+  // the current segment, read from the plan once per step / segment
+  int j, n_seg, s_pos, s_len, s_row, shift;
   int vis_lo, vis_hi, full_lo, full_hi;
+
+  __device__ void enter_seg() {
+    if (sg < n_seg) {
+      s_pos = pl->seg[j][sg].pos;
+      s_len = pl->seg[j][sg].len;
+      s_row = pl->seg[j][sg].buf_row;
+    }
+  }
+  __device__ void enter_step() {
+    j = r - t;
+    if (j < 0) j += P;
+    n_seg = pl->nseg[j];
+    shift = (striped && j > r) ? 1 : 0;
+    sg = tl = 0;
+    enter_seg();
+  }
 
   __device__ void init(const cp_bwd_plan& p, const Own& own) {
     pl = &p;
     r = own.rank;
     row0 = own.grp_row0;
+    P = p.P;
+    t_end = p.t_end;
+    striped = p.striped != 0;
     t = p.t_begin;
-    sg = tl = 0;
+    if (t < t_end) enter_step();
     const int qa = own.pos0, qb = own.pos0 + own.valid - 1;
     const bool docs = p.n_docs > 0;
     vis_lo = docs ? bdoc_start(p.cu_seqlens, p.n_docs, qa) : kNoLo;
@@ -170,37 +194,34 @@ struct DqIter {
   }
 
   __device__ bool next(KvTile& out) {
-    const int P = pl->P;
-    while (t < pl->t_end) {
-      const int j = ((r - t) % P + P) % P;
-      if (sg >= pl->nseg[j]) {
-        ++t;
-        sg = tl = 0;
+    while (t < t_end) {
+      if (sg >= n_seg) {
+        if (++t < t_end) enter_step();
         continue;
       }
-      const cp_seg& s = pl->seg[j][sg];
       const int off = tl * 128;
-      if (off >= s.len) {
+      if (off >= s_len) {
         ++sg;
         tl = 0;
+        enter_seg();
         continue;
       }
-      const int shift = (pl->striped && j > r) ? 1 : 0;
-      const int ka = s.pos + shift + off;
+      const int ka = s_pos + shift + off;
       if (ka > vis_hi) {  // positions grow along a segment
         ++sg;
         tl = 0;
+        enter_seg();
         continue;
       }
       if (ka + 127 < vis_lo) {  // keys of earlier documents: jump to the first visible tile
-        tl = (vis_lo - s.pos - shift) / 128;
+        tl = (vis_lo - s_pos - shift) / 128;
         continue;
       }
       ++tl;
-      const int valid = min(128, s.len - off);
+      const int valid = min(128, s_len - off);
       const int kb = ka + valid - 1;
       if (kb >= vis_lo && ka <= vis_hi) {
-        out.buf_row = row0 + s.buf_row + off;
+        out.buf_row = row0 + s_row + off;
         out.pos = ka;
         out.valid = valid;
         out.full = valid == 128 && ka >= full_lo && kb <= full_hi;
@@ -561,16 +582,43 @@ struct QTile {
 struct KvIter {
   const cp_bwd_plan* pl;
   int j, hk, g, t, sg, tl, row0;
+  int P, t_begin, t_end, group;
+  bool striped_causal;
+  // the current ring step's rank r = (j + t) mod P, its segment count and
+  // the current segment, read from the plan once per step / segment
+  int r, n_seg, s_pos, s_len, s_row, shift;
   int ka0, kb0;                    // own positions without the striped shift
   int lo0, hi0, flo0, fhi0;        // windows of admitted query positions
+
+  __device__ void enter_seg() {
+    if (sg < n_seg) {
+      s_pos = pl->seg[r][sg].pos;
+      s_len = pl->seg[r][sg].len;
+      s_row = pl->seg[r][sg].buf_row;
+    }
+  }
+  __device__ void enter_step() {
+    r = j + t;
+    if (r >= P) r -= P;
+    n_seg = pl->nseg[r];
+    shift = (striped_causal && j > r) ? 1 : 0;
+    sg = tl = 0;
+    enter_seg();
+  }
 
   __device__ void init(const cp_bwd_plan& p, const Own& own, int kv_head) {
     pl = &p;
     j = own.rank;
     hk = kv_head;
     row0 = own.grp_row0;
+    P = p.P;
+    t_begin = p.t_begin;
+    t_end = p.t_end;
+    group = p.hq / p.hkv;
+    striped_causal = p.striped && p.causal;
     g = sg = tl = 0;
     t = p.t_begin;
+    if (t < t_end) enter_step();
     ka0 = own.pos0;
     kb0 = own.pos0 + own.valid - 1;
     const bool docs = p.n_docs > 0;
@@ -582,44 +630,40 @@ struct KvIter {
   }
 
   __device__ bool next(QTile& out) {
-    const int P = pl->P;
-    const int group = pl->hq / pl->hkv;
     while (g < group) {
-      if (t >= pl->t_end) {
+      if (t >= t_end) {
         ++g;
-        t = pl->t_begin;
-        sg = tl = 0;
+        t = t_begin;
+        if (t < t_end) enter_step();
         continue;
       }
-      const int r = (j + t) % P;
-      if (sg >= pl->nseg[r]) {
-        ++t;
-        sg = tl = 0;
+      if (sg >= n_seg) {
+        if (++t < t_end) enter_step();
         continue;
       }
-      const cp_seg& s = pl->seg[r][sg];
       const int off = tl * 128;
-      if (off >= s.len) {
+      if (off >= s_len) {
         ++sg;
         tl = 0;
+        enter_seg();
         continue;
       }
-      const int shift = (pl->striped && pl->causal && j > r) ? 1 : 0;
-      const int qa = s.pos + off;
+      const int qa = s_pos + off;
       if (qa > hi0) {  // positions grow along a segment
         ++sg;
         tl = 0;
+        enter_seg();
         continue;
       }
       if (qa + 127 < lo0 + shift) {  // queries before the key (or its document): jump over them
-        tl = (lo0 + shift - s.pos) / 128;
+        tl = (lo0 + shift - s_pos) / 128;
         continue;
       }
       ++tl;
-      const int valid = min(128, s.len - off);
+      const int valid = min(128, s_len - off);
       const int qb = qa + valid - 1;
       if (qb >= lo0 + shift && qa <= hi0) {
-        out.buf_row = row0 + s.buf_row + off;
+        out.buf_row = row0 + s_row + off;
         out.pos = qa;
         out.valid = valid;
         out.h = hk * group + g;

@@ -77,33 +77,41 @@ struct KTile {
 // copy, so all of them see the same sequence without communicating.
 struct KIter {
   const cp_pair_desc* pd;
-  int seg, t;
+  int seg, t, nk;
+  int len, pos, row;  // the current segment, read from the plan once per segment
   int vis_lo[2], vis_hi[2];
   int lo_min;  // first position visible to either live sub-tile
   bool alive[2];
 
+  __device__ void enter(int s) {
+    seg = s;
+    t = 0;
+    if (s < nk) {
+      len = pd->k[s].len;
+      pos = pd->k[s].pos;
+      row = pd->k[s].buf_row;
+    }
+  }
+
   __device__ bool next(KTile& out) {
-    while (seg < pd->nk) {
-      const int len = pd->k[seg].len;
+    while (seg < nk) {
       const int off = t * CP_KV_TILE;
       if (off >= len) {
-        ++seg;
-        t = 0;
+        enter(seg + 1);
         continue;
       }
-      const int ka = pd->k[seg].pos + off;
+      const int ka = pos + off;
       // Positions grow along a segment: once past both causal limits, the
       // rest of the segment is masked.
       if ((!alive[0] || ka > vis_hi[0]) && (!alive[1] || ka > vis_hi[1])) {
-        ++seg;
-        t = 0;
+        enter(seg + 1);
         continue;
       }
       // Tiles that end before both windows start (keys of earlier documents)
       // are jumped over in one step, to the tile holding the first visible
       // position.
       if (ka + CP_KV_TILE - 1 < lo_min) {
-        t = (lo_min - pd->k[seg].pos) / CP_KV_TILE;
+        t = (lo_min - pos) / CP_KV_TILE;
         continue;
       }
       ++t;
@@ -112,7 +120,7 @@ struct KIter {
       const bool l0 = alive[0] && kb >= vis_lo[0] && ka <= vis_hi[0];
       const bool l1 = alive[1] && kb >= vis_lo[1] && ka <= vis_hi[1];
       if (l0 || l1) {
-        out.buf_row = pd->k[seg].buf_row + off;
+        out.buf_row = row + off;
         out.pos = ka;
         out.valid = valid;
         out.live0 = l0;
@@ -201,14 +209,14 @@ __device__ __forceinline__ void decode_item(const cp_attn_plan& plan, const int3
 
 __device__ __forceinline__ void make_iter(const Item& it, KIter& ki) {
   ki.pd = it.pd;
-  ki.seg = 0;
-  ki.t = 0;
+  ki.nk = it.pd->nk;
   for (int t = 0; t < 2; ++t) {
     ki.vis_lo[t] = it.vis_lo[t];
     ki.vis_hi[t] = it.vis_hi[t];
     ki.alive[t] = it.alive[t];
   }
   ki.lo_min = min(it.alive[0] ? it.vis_lo[0] : INT_MAX, it.alive[1] ? it.vis_lo[1] : INT_MAX);
+  ki.enter(0);
 }
 
 template <int DH>

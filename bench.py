@@ -68,11 +68,11 @@ BWD_SUITE = ["ring_contig_32k", "varlen_zigzag_128k"]
 # repeated.  Filled from the profiles/ summaries.
 ATTN_TRAFFIC = {
     # profiles/attn_fwd_kernel_dram_ring_workloads.md (one-pass DRAM read + write per launch)
-    ("0f2224ea9ddfd474", "ring_contig_32k"): 2.1437e9,
-    ("0f2224ea9ddfd474", "ring_zigzag_64k"): 9.7940e9,
-    ("0f2224ea9ddfd474", "varlen_zigzag_128k"): 9.9621e9,
-    ("0f2224ea9ddfd474", "ring_striped_64k"): 13.6606e9,
-    ("0f2224ea9ddfd474", "ulysses_gqa_128k"): 6.7052e9,
+    ("3f5eba916fea743e", "ring_contig_32k"): 2.1446e9,
+    ("3f5eba916fea743e", "ring_zigzag_64k"): 9.7936e9,
+    ("3f5eba916fea743e", "varlen_zigzag_128k"): 9.9624e9,
+    ("3f5eba916fea743e", "ring_striped_64k"): 13.6513e9,
+    ("3f5eba916fea743e", "ulysses_gqa_128k"): 6.7032e9,
 }
 
 

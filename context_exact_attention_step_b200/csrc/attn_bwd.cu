@@ -704,7 +704,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   float* sVec = reinterpret_cast<float*>(sStage + C::kStages * C::kStageBytes);
   uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sVec) + C::kStages * C::kVecBytes);
   const int B_KV = 0, B_FULL = 1, B_EMPTY = 1 + C::kStages, B_S = 1 + 2 * C::kStages, B_DP = B_S + 1,
-            B_P = B_DP + 1, B_DS = B_P + 1, B_ACC = B_DS + 1, B_DRAIN = B_ACC + 1, B_COUNT = B_DRAIN + 1;
+            B_P = B_DP + 1, B_DS = B_P + 1, B_DPR = B_DS + 1, B_ACC = B_DPR + 1, B_DRAIN = B_ACC + 1,
+            B_COUNT = B_DRAIN + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + B_COUNT);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   auto bar = [&](int i) { return smem_addr(bars + i); };
@@ -722,6 +723,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(bar(B_DP), 1);
     mbar_init(bar(B_P), 8);  // one arrive per element-wise warp
     mbar_init(bar(B_DS), 8);
+    mbar_init(bar(B_DPR), 8);  // dP^T read out of TMEM by every element-wise warp
     mbar_init(bar(B_ACC), 1);
     mbar_init(bar(B_DRAIN), 1);
     *abort_flag = 0;
@@ -865,14 +867,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!(ok = mbar_wait_warp(bar(B_P), i & 1u, abort_flag, err, kWaitNs))) break;
       tc_fence_after();
       issue_acc(C::kColDV, col_r(i) + 0, col_r(i) + 96, smem_addr(stage_do(s)), i > 0);
-      if (!(ok = mbar_wait_warp(bar(B_DS), i & 1u, abort_flag, err, kWaitNs))) break;
-      tc_fence_after();
       if (hn) {
+        // S^T(i+1) goes where dP^T(i) lives: issued as soon as every
+        // element-wise warp has read dP^T(i), while they still form dS^T(i)
+        if (!(ok = mbar_wait_warp(bar(B_DPR), i & 1u, abort_flag, err, kWaitNs))) break;
         if (!(ok = mbar_wait_warp(bar(B_FULL + slot_of(i + 1)), ph_of(i + 1), abort_flag, err, kWaitNs))) break;
         tc_fence_after();
         issue_ss(col_r(i + 1), sk, smem_addr(stage_q(slot_of(i + 1))));
         tc_commit_elect(bar(B_S));
       }
+      if (!(ok = mbar_wait_warp(bar(B_DS), i & 1u, abort_flag, err, kWaitNs))) break;
+      tc_fence_after();
       issue_acc(C::kColDK, col_r(i) + 32, col_r(i) + 64, smem_addr(stage_q(s)), i > 0);
       tc_commit_elect(bar(B_EMPTY + s));
       if (hn) {
@@ -973,6 +978,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_ld32(tD, *reinterpret_cast<uint32_t(*)[32]>(&d[0]));
         tmem_ld32(tD + 32, *reinterpret_cast<uint32_t(*)[32]>(&d[32]));
         tc_wait_ld();
+        // dP^T(i) is in registers: its TMEM columns may take S^T(i+1)
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_DPR));
         uint32_t w[32];
 #pragma unroll
         for (int i4 = 0; i4 < 16; ++i4) {

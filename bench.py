@@ -67,7 +67,9 @@ BWD_SUITE = ["ring_contig_32k", "varlen_zigzag_128k"]
 # change makes the entry stale and the line reports null until the capture is
 # repeated.  Filled from the profiles/ summaries.
 ATTN_TRAFFIC = {
-    # profiles/attn_fwd_kernel_dram_ring_workloads.md (one-pass DRAM read + write per launch)
+    # profiles/attn_fwd_kernel_dram_ring_workloads.md (one-pass DRAM read + write per launch), taken
+    # on the source before the MMA descriptors were derived by offset: the current source reports
+    # null until the capture is repeated on it.
     ("3f5eba916fea743e", "ring_contig_32k"): 2.1446e9,
     ("3f5eba916fea743e", "ring_zigzag_64k"): 9.7936e9,
     ("3f5eba916fea743e", "varlen_zigzag_128k"): 9.9624e9,

@@ -349,21 +349,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // D[col] = A B^T over dh: A (Q or dO, bf16 in TMEM at column acol, 8
     // columns per K-step of 16) times a K-major 128-row key/value tile
     auto issue_ss = [&](uint32_t dcol, uint32_t acol, uint32_t b_base) {
+      const uint64_t b0 = sdesc_sw128(b_base, 16, 1024);
 #pragma unroll
       for (int kk = 0; kk < DH / 16; ++kk) {
-        const uint32_t box = kk >> 2, koff = (kk & 3) * 32;
-        const uint64_t b = sdesc_sw128(b_base + box * T::kBoxBytes + koff, 16, 1024);
-        tc_mma_ts_elect(tmem + dcol, tmem + acol + kk * 8, b, idesc_ss, kk > 0 ? 1u : 0u);
+        const uint32_t off = (kk >> 2) * T::kBoxBytes + (kk & 3) * 32;
+        tc_mma_ts_elect(tmem + dcol, tmem + acol + kk * 8, sdesc_add(b0, off), idesc_ss, kk > 0 ? 1u : 0u);
       }
     };
     // dQ += dS K: A = dS (bf16 in TMEM, 128 keys as 8 K-steps of 16; keys
     // 0-63 at dcol, keys 64-127 at dcol + 64), B = the K tile read MN-major
     auto issue_dq = [&](uint32_t dcol, uint32_t kbase, bool acc) {
+      const uint64_t b0 = sdesc_sw128(kbase, T::kBoxBytes, 1024);
 #pragma unroll
       for (int kk = 0; kk < 128 / 16; ++kk) {
         const uint32_t acol = kk < 4 ? dcol + kk * 8 : dcol + 64 + (kk - 4) * 8;
-        const uint64_t b = sdesc_sw128(kbase + kk * 2048, T::kBoxBytes, 1024);
-        tc_mma_ts_elect(tmem + C::kColQ, tmem + acol, b, idesc_dq, (acc || kk > 0) ? 1u : 0u);
+        tc_mma_ts_elect(tmem + C::kColQ, tmem + acol, sdesc_add(b0, kk * 2048), idesc_dq, (acc || kk > 0) ? 1u : 0u);
       }
     };
     auto kslot = [&](int j) { return (2 * j) % C::kStages; };
@@ -822,23 +822,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     constexpr uint32_t idesc_acc = idesc_bf16_f32(128, DH, true);
     const uint32_t sk = smem_addr(sK), sv = smem_addr(sV);
     auto issue_ss = [&](uint32_t dcol, uint32_t a_base, uint32_t b_base) {
+      const uint64_t a0 = sdesc_sw128(a_base, 16, 1024);
+      const uint64_t b0 = sdesc_sw128(b_base, 16, 1024);
 #pragma unroll
       for (int kk = 0; kk < DH / 16; ++kk) {
-        const uint32_t box = kk >> 2, koff = (kk & 3) * 32;
-        const uint64_t a = sdesc_sw128(a_base + box * T::kBoxBytes + koff, 16, 1024);
-        const uint64_t b = sdesc_sw128(b_base + box * T::kBoxBytes + koff, 16, 1024);
-        tc_mma_ss_elect(tmem + dcol, a, b, idesc_ss, kk > 0 ? 1u : 0u);
+        const uint32_t off = (kk >> 2) * T::kBoxBytes + (kk & 3) * 32;
+        tc_mma_ss_elect(tmem + dcol, sdesc_add(a0, off), sdesc_add(b0, off), idesc_ss, kk > 0 ? 1u : 0u);
       }
     };
     // D[dcol] += A (bf16 in TMEM, 128 query rows as 8 K-steps of 16) x B (a
     // 128-row query-side tile read MN-major).  The A columns of K-steps 0-3
     // (queries 0-63) start at lo_col, those of K-steps 4-7 at hi_col.
     auto issue_acc = [&](uint32_t dcol, uint32_t lo_col, uint32_t hi_col, uint32_t b_base, bool acc) {
+      const uint64_t b0 = sdesc_sw128(b_base, T::kBoxBytes, 1024);
 #pragma unroll
       for (int kk = 0; kk < 128 / 16; ++kk) {
         const uint32_t acol = kk < 4 ? lo_col + kk * 8 : hi_col + (kk - 4) * 8;
-        const uint64_t b = sdesc_sw128(b_base + kk * 2048, T::kBoxBytes, 1024);
-        tc_mma_ts_elect(tmem + dcol, tmem + acol, b, idesc_acc, (acc || kk > 0) ? 1u : 0u);
+        tc_mma_ts_elect(tmem + dcol, tmem + acol, sdesc_add(b0, kk * 2048), idesc_acc, (acc || kk > 0) ? 1u : 0u);
       }
     };
     auto slot_of = [&](int i) { return i % C::kStages; };

@@ -328,21 +328,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t sq_base = smem_addr(sQ);
     const uint32_t skv_base = smem_addr(sKV);
     auto issue_s = [&](int t, int slot) {
+      const uint64_t a0 = sdesc_sw128(sq_base + t * C::kBoxes * C::kBoxBytes, 16, 1024);
+      const uint64_t b0 = sdesc_sw128(skv_base + slot * C::kTileBytes, 16, 1024);
 #pragma unroll
       for (int kk = 0; kk < DH / 16; ++kk) {
-        const uint32_t box = kk >> 2, koff = (kk & 3) * 32;
-        const uint64_t a = sdesc_sw128(sq_base + (t * C::kBoxes + box) * C::kBoxBytes + koff, 16, 1024);
-        const uint64_t b = sdesc_sw128(skv_base + slot * C::kTileBytes + box * C::kBoxBytes + koff, 16, 1024);
-        tc_mma_ss_elect(tmem + C::col_s(t), a, b, idesc_qk, kk > 0 ? 1u : 0u);
+        const uint32_t off = (kk >> 2) * C::kBoxBytes + (kk & 3) * 32;
+        tc_mma_ss_elect(tmem + C::col_s(t), sdesc_add(a0, off), sdesc_add(b0, off), idesc_qk, kk > 0 ? 1u : 0u);
       }
     };
     // O_t += P_t V over the 64 keys of half h of the tile
     auto issue_pv_half = [&](int t, int slot, int h, bool acc) {
+      const uint64_t b0 = sdesc_sw128(skv_base + slot * C::kTileBytes, C::kBoxBytes, 1024);
 #pragma unroll
       for (int k4 = 0; k4 < CP_KV_TILE / 32; ++k4) {
         const int kk = h * (CP_KV_TILE / 32) + k4;
-        const uint64_t b = sdesc_sw128(skv_base + slot * C::kTileBytes + kk * 2048, C::kBoxBytes, 1024);
-        tc_mma_ts_elect(tmem + C::col_o(t), tmem + C::col_s(t) + kk * 8, b, idesc_pv, (acc || kk > 0) ? 1u : 0u);
+        tc_mma_ts_elect(tmem + C::col_o(t), tmem + C::col_s(t) + kk * 8, sdesc_add(b0, kk * 2048), idesc_pv,
+                        (acc || kk > 0) ? 1u : 0u);
       }
     };
     // P_t is released in two halves: the first half's MMAs run while the

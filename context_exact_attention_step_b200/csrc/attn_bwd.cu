@@ -237,6 +237,7 @@ struct DqCfg {
   using T = BwdTile<DH>;
   static constexpr int kStages = DH == 128 ? 4 : 8;
   static constexpr int kSmemBytes = 1024 + 2 * T::kTileBytes + kStages * T::kTileBytes + 256;
+  static_assert(kSmemBytes <= kMaxSmemPerCta, "dQ kernel exceeds the shared memory of a CTA");
   // TMEM: S | dP (dS is written over it) | dQ | Q and dO as the A operands of
   // S = Q K^T and dP = dO V^T, copied in once so that these MMAs read only
   // K and V from shared memory
@@ -684,6 +685,7 @@ struct DkvCfg {
   static constexpr int kVecBytes = 2 * 128 * 4;          // -LSE*log2(e) and D of the 128 query rows
   static constexpr int kSmemBytes =
       1024 + 2 * T::kTileBytes + kStages * kStageBytes + kStages * kVecBytes + 256;
+  static_assert(kSmemBytes <= kMaxSmemPerCta, "dK/dV kernel exceeds the shared memory of a CTA");
   // TMEM: two 128-column buffers (S^T with P^T and dS^T written over it, and
   // dP^T, alternating per query tile) | dV | dK
   static constexpr uint32_t kColDV = 256, kColDK = 256 + DH;

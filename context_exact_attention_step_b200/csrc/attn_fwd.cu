@@ -61,6 +61,7 @@ struct AttnCfg {
   static constexpr int kQBytes = 2 * kTileBytes;
   static constexpr int kBarBytes = 256;
   static constexpr int kSmemBytes = 1024 + kQBytes + kStages * kTileBytes + kBarBytes + kCuSmem * 4;
+  static_assert(kSmemBytes <= kMaxSmemPerCta, "forward kernel exceeds the shared memory of a CTA");
   static constexpr uint32_t kTmemCols = 512;
   // TMEM column of the S/P tile and of the O accumulator of sub-tile t
   __device__ static constexpr uint32_t col_s(int t) { return (uint32_t)t * 128u; }

@@ -161,6 +161,11 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
 // address field is linear in the address, and shared-window addresses stay
 // below 2^18, so the 14-bit field never carries into the fields above it
 // (one 32-bit add per MMA instead of rebuilding the descriptor).
+// Dynamic shared memory a CTA may request on sm_100 (227 KB): every shared
+// address a kernel forms stays below 2^18, the precondition of sdesc_add.
+constexpr int kMaxSmemPerCta = 227 * 1024;
+static_assert(kMaxSmemPerCta < (1 << 18), "shared addresses must fit the descriptor's 14-bit start field");
+
 __device__ __forceinline__ uint64_t sdesc_add(uint64_t desc, uint32_t byte_off) {
   uint32_t lo, hi;
   asm("mov.b64 {%0, %1}, %2;" : "=r"(lo), "=r"(hi) : "l"(desc));

@@ -32,8 +32,10 @@
 //
 // CTA layout of both tensor-core kernels (384 threads, one CTA per SM):
 //   warp 0      TMA producer
-//   warp 1      tcgen05.mma issuer (one elected lane) and TMEM owner
-//   warps 2-3   idle
+//   warp 1      tcgen05.mma issuer (whole warp converged, an elected lane
+//               issues each MMA and commit) and TMEM owner
+//   warps 2-3   no work: they complete the control warpgroup, whose four
+//               warps give back registers together (setmaxnreg)
 //   warps 4-7   element-wise stage, columns 0-63 of every tile, one own row
 //               per thread (TMEM lane)
 //   warps 8-11  element-wise stage, columns 64-127 of the same rows
